@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the H-BitLinear forward (BitNet v2) on B200.
+
+Workload (one step): the decode-shaped o_proj H-BitLinear, M=16 tokens,
+K=N=4096, W1.58A4 with the Hadamard on, run once for each of 64 distinct
+packed weight sets (64 x 4 MiB = 256 MiB, larger than the 126 MB L2, so every
+forward streams its weights from HBM). The 64 forwards of a step are captured
+in one CUDA graph. value = tokens/s over the whole job (tokens = M per forward).
+
+Also reported: the dominant kernel's roofline fraction (CUDA-event duration
+of that kernel, algorithmic bytes), the same metric end to end through the C
+ABI with the host<->device copies in the timed region, SM clocks during the
+run, the CPU oracle on a bounded sample, and secondary configurations.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same step on its own GPU (token-sharded
+replicas, weak scaling, no collective in the data path); rank 0 prints one
+JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "H-BitLinear fwd TOPS & tokens/s (W1.58A4) + % of HBM/tensor roofline"
+LAYERS = 64
+HEAD = dict(M=16, K=4096, N=4096, act_bits=4, use_hadamard=1)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "hadamard_bit_quant_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernels."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{workload}/{kernel}")
+    if not e or e.get("csrc_sha") != csrc_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def headline_workload_name():
+    return (f"decode_oproj M={HEAD['M']} K={HEAD['K']} N={HEAD['N']} W1.58A{HEAD['act_bits']} "
+            f"H{'on' if HEAD['use_hadamard'] else 'off'}, {LAYERS} weight sets per step")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for k, nm in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                          ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+def cpu_oracle_baseline(X, W, case, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the headline batch (rank 0, N=1)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    Xn = X.double().numpy()
+    a, T = oracle.weight_quant(W.numpy())          # offline weight packing: not timed
+    oracle.forward(Xn[:1], T, a, case["act_bits"], case["use_hadamard"])   # builds H once
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.forward(Xn, T, a, case["act_bits"], case["use_hadamard"])
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n * case["M"] / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} full oracle forwards of the M={case['M']} headline batch "
+                      f"(explicit O(K^2) fp64 Hadamard, fp64 quantiser, exact GEMM) in {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    import oracle
+    from hadamard_bit_quant_b200 import inputs
+    case = [c for c in inputs.decode_oproj_cases((HEAD["M"],), (HEAD["act_bits"],))][0]
+    X = case.make_x().double().numpy()
+    a, T = oracle.weight_quant(case.make_w().numpy())
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = len(os.sched_getaffinity(0))
+    # one step = the oracle forward of one token of the batch (a bounded sample)
+    def step(i):
+        oracle.forward(X[i % case.M:i % case.M + 1], T, a, case.act_bits, case.use_hadamard)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    val = args.steps / dt
+    cfg = {"workload": headline_workload_name(), "M": case.M, "K": case.K, "N": case.N,
+           "act_bits": case.act_bits, "use_hadamard": case.use_hadamard}
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "impl": "reference",
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": "one token of the batch per step through the oracle forward"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def capture_step(torch, hbl, X, Wpks, wsc, Y, ws, case, Xh=None, Yh=None):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=s):
+        for Wpk in Wpks:
+            if Xh is not None:
+                X.copy_(Xh, non_blocking=True)
+            hbl.hbl_forward_ws(X, case["M"], case["K"], case["N"], Wpk, wsc, case["act_bits"],
+                               case["use_hadamard"], Y, ws, ws.numel())
+            if Yh is not None:
+                Yh.copy_(Y, non_blocking=True)
+    return g
+
+
+def timed_replays(torch, dist, g, warmup, steps, world):
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+KERNEL_BYTES = {
+    # algorithmic bytes per launch (what the step must move), per kernel kind
+    "gemm_mma": lambda M, K, N: N * K / 4 + M * K + 2 * M * N + 4 * M + 4,
+    "fwht_quant": lambda M, K, N: M * (2 * K + K + 8),
+    "quant_rows": lambda M, K, N: M * (2 * K + K + 8),
+    "dequant_store": lambda M, K, N: 4 * M * N + 2 * M * N + 8 * M,
+}
+
+
+def profile_kernels(torch, hbl, X, Wpks, wsc, Y, ws, case, reps):
+    """Per-kernel CUDA-event durations of the forward, weights cold (L2 flushed before each)."""
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    hbl.hbl_profile_enable(1)
+    for r in range(reps):
+        flush.zero_()
+        hbl.hbl_forward_ws(X, case["M"], case["K"], case["N"], Wpks[r % len(Wpks)], wsc, case["act_bits"],
+                           case["use_hadamard"], Y, ws, ws.numel())
+    torch.cuda.synchronize()
+    tab = hbl.profile_table()
+    hbl.hbl_profile_enable(0)
+    del flush
+    return {k: {"launches": n, "ms_per_launch": ms / max(n, 1)} for k, (n, ms) in tab.items()}
+
+
+def roofline_of(prof, case, peaks, peak_kind, workload):
+    ours = {k: v for k, v in prof.items() if k in KERNEL_BYTES}
+    dom = max(ours, key=lambda k: ours[k]["ms_per_launch"] * ours[k]["launches"])
+    b = KERNEL_BYTES[dom](case["M"], case["K"], case["N"])
+    t = ours[dom]["ms_per_launch"] * 1e-3
+    ach = b / t / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+            "traffic": traffic_for(dom, workload), "kernel": dom, "bytes_per_launch": b,
+            "launch_us": t * 1e6, "peak_source": f"{peak_kind} hbm_gbs"}
+
+
+def secondary(torch, hbl, layer, inputs):
+    """Other decode shapes (graph of 64 forwards, 20 replays) and the prefill config."""
+    out = {}
+    for case in inputs.decode_oproj_cases():
+        if case.M == HEAD["M"] and case.act_bits == HEAD["act_bits"]:
+            continue
+        c = dict(M=case.M, K=case.K, N=case.N, act_bits=case.act_bits, use_hadamard=case.use_hadamard)
+        X = case.make_x().cuda()
+        Wpk, wsc = layer.pack_weights(case.make_w().cuda())
+        Wpks = [Wpk] + [Wpk.clone() for _ in range(LAYERS - 1)]
+        Y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device="cuda")
+        ws = layer.workspace(case.M, case.K, case.N, "cuda")
+        hbl.hbl_forward_ws(X, case.M, case.K, case.N, Wpk, wsc, case.act_bits, case.use_hadamard, Y, ws, ws.numel())
+        g = capture_step(torch, hbl, X, Wpks, wsc, Y, ws, c)
+        ms = timed_replays(torch, None, g, 3, 20, 1) / (20 * LAYERS)
+        out[f"decode M={case.M} a{case.act_bits}"] = {
+            "us_per_forward": ms * 1e3, "tokens_per_s": case.M / (ms * 1e-3),
+            "weight_GBps": case.N * case.K / 4 / (ms * 1e-3) / 1e9}
+        del g, Wpks
+    case = inputs.prefill_down_case()
+    X = case.make_x().cuda()
+    Wpk, wsc = layer.pack_weights(case.make_w().cuda())
+    Y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device="cuda")
+    ws = layer.workspace(case.M, case.K, case.N, "cuda")
+    c = dict(M=case.M, K=case.K, N=case.N, act_bits=case.act_bits, use_hadamard=case.use_hadamard)
+    hbl.hbl_forward_ws(X, case.M, case.K, case.N, Wpk, wsc, case.act_bits, case.use_hadamard, Y, ws, ws.numel())
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    times = []
+    for _ in range(5):
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        hbl.hbl_forward_ws(X, case.M, case.K, case.N, Wpk, wsc, case.act_bits, case.use_hadamard, Y, ws, ws.numel())
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    prof = profile_kernels(torch, hbl, X, [Wpk], wsc, Y, ws, c, 3)
+    ms = statistics.median(times)
+    ops = 2.0 * case.M * case.N * case.K
+    gemm_ms = prof.get("gemm_mma", {}).get("ms_per_launch")
+    out["prefill M=4096 K=16384 N=4096 a4"] = {
+        "ms_forward": ms, "tokens_per_s": case.M / (ms * 1e-3), "TOPS": ops / (ms * 1e-3) / 1e12,
+        "gemm_ms": gemm_ms, "gemm_TOPS": (ops / (gemm_ms * 1e-3) / 1e12) if gemm_ms else None,
+        "kernels": prof}
+    return out
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from hadamard_bit_quant_b200 import build, hbl, inputs, layer
+    if not os.path.exists(os.path.join(ROOT, "hadamard_bit_quant_b200", "libhbl.so")):
+        build.build()
+    hbl.lib()
+    peaks, peak_kind = load_peaks()
+    case = [c for c in inputs.decode_oproj_cases((HEAD["M"],), (HEAD["act_bits"],))][0]
+    c = dict(HEAD)
+    Xc, Wc = case.make_x(), case.make_w()
+    X = Xc.cuda()
+    Wpk, wsc = layer.pack_weights(Wc.cuda())
+    Wpks = [Wpk] + [Wpk.clone() for _ in range(LAYERS - 1)]
+    Y = torch.empty(c["M"], c["N"], dtype=torch.bfloat16, device="cuda")
+    ws = layer.workspace(c["M"], c["K"], c["N"], "cuda")
+    # eager call first: library init (device probe, kernel attributes) happens outside capture
+    hbl.hbl_forward_ws(X, c["M"], c["K"], c["N"], Wpk, wsc, c["act_bits"], c["use_hadamard"], Y, ws, ws.numel())
+    torch.cuda.synchronize()
+    g = capture_step(torch, hbl, X, Wpks, wsc, Y, ws, c)
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    clocks.start()
+    ms = timed_replays(torch, dist, g, args.warmup, args.steps, world)
+    clk = clocks.stop()
+    tokens = world * args.steps * LAYERS * c["M"]
+    value = tokens / (ms * 1e-3)
+    ops_per_step = 2.0 * LAYERS * c["M"] * c["N"] * c["K"]
+
+    # e2e: same step with the H2D copy of each forward's input and the D2H copy of its output
+    Xh = Xc.pin_memory()
+    Yh = torch.empty(c["M"], c["N"], dtype=torch.bfloat16).pin_memory()
+    g2 = capture_step(torch, hbl, X, Wpks, wsc, Y, ws, c, Xh=Xh, Yh=Yh)
+    ms_e2e = timed_replays(torch, dist, g2, args.warmup, args.steps, world)
+    e2e = {"value": tokens / (ms_e2e * 1e-3), "unit": "tokens/s",
+           "h2d_bytes_per_step": LAYERS * Xh.numel() * 2, "d2h_bytes_per_step": LAYERS * Yh.numel() * 2}
+
+    prof = profile_kernels(torch, hbl, X, Wpks, wsc, Y, ws, c, 64)
+    launches_per_forward = sum(v["launches"] for k, v in prof.items() if k != "memset_acc") / 64
+    roof = roofline_of(prof, c, peaks, peak_kind, "decode_oproj_m16")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": headline_workload_name(), "M": c["M"], "K": c["K"], "N": c["N"],
+                   "act_bits": c["act_bits"], "use_hadamard": c["use_hadamard"], "layers_per_step": LAYERS,
+                   "tokens_per_step_per_gpu": LAYERS * c["M"],
+                   "l2": "inputs larger than L2: 64 packed weight sets (256 MiB) rotate within each step",
+                   "parallelism": f"dp{world} (token-sharded replicas, no collective)", "graph": True},
+        "tops": ops_per_step * args.steps * world / (ms * 1e-3) / 1e12,
+        "roofline": roof,
+        "kernels": prof,
+        "e2e": e2e,
+        "gpu_launches": int(round(launches_per_forward * LAYERS * args.steps)),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_extras:
+        try:
+            line["secondary"] = secondary(torch, hbl, layer, inputs)
+        except Exception as ex:  # secondary numbers are optional context
+            line["secondary"] = {"error": repr(ex)}
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_oracle_baseline(Xc, Wc, c)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g, g2
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,339 @@
+// Online Hadamard transform + per-token activation quantiser.
+//
+// BitNet v2 architecture walkthrough, section 3.4:
+//   * "The Hadamard Transformation", Eq. 3-6: X_r = H_m x, Sylvester H_m with
+//     2^(-m/2) scaling, computed by the fast Walsh-Hadamard transform
+//     (log2 K butterfly stages).
+//   * "Activation Quantization", Eq. 7 (INT8, absmax/127) and Eq. 8 (INT4,
+//     absmean/sqrt7), per token, RoundClip with round-half-to-even.
+//
+// Kernel structure (one token per T = K/E threads, E = 2^G values per thread):
+// the log2 K butterfly stages commute, so they are grouped into passes of G
+// index bits, processed top-down. In a pass that owns bits [lo, lo+G), thread
+// t holds the E values whose indices differ only in those bits, and the
+// butterflies run in registers. Between passes the values are exchanged
+// through shared memory (an XOR swizzle keeps both access patterns free of
+// bank conflicts). The first pass owns the top bits, so its loads are
+// coalesced across threads; the last pass owns bits [0, G), so each thread
+// ends with E consecutive values and stores E consecutive codes.
+#pragma once
+#include "hbl_common.cuh"
+
+namespace hbl {
+
+enum QuantMode { kModeInt4 = 0, kModeInt8 = 1, kModeF32 = 2 };
+
+template <int LOG_K, int G>
+struct FwhtCfg {
+  static constexpr int K = 1 << LOG_K;
+  static constexpr int E = 1 << G;
+  static constexpr int T = K / E;                       // threads per token
+  static constexpr int TPC = T >= 128 ? 1 : 128 / T;    // tokens per CTA
+  static constexpr int THREADS = T * TPC;
+  static constexpr int P = (LOG_K + G - 1) / G;         // passes
+  static constexpr int WARPS_PER_TOKEN = T >= 32 ? T / 32 : 1;
+  static constexpr size_t SMEM = (size_t)TPC * K * sizeof(float);
+};
+
+template <int G>
+HBL_DEVINL int pass_index(int t, int j, int lo) {
+  const int low = t & ((1 << lo) - 1);
+  const int high = t >> lo;
+  return low | (j << lo) | (high << (lo + G));
+}
+
+template <int G>
+HBL_DEVINL int swz(int idx) { return idx ^ ((idx >> G) & 31); }
+
+// Sum / max over the T threads of one token. Threads of a token are T
+// consecutive lanes (T < 32) or T/32 whole warps (T >= 32). `red` holds one
+// slot per warp. Deterministic (fixed reduction order).
+template <int T, int WPT, bool IS_MAX>
+HBL_DEVINL float token_reduce_f(float x, float* red, int token_sub) {
+  constexpr int W = T < 32 ? T : 32;
+#pragma unroll
+  for (int off = W / 2; off > 0; off >>= 1) {
+    float o = __shfl_xor_sync(0xffffffffu, x, off);
+    x = IS_MAX ? fmaxf(x, o) : x + o;
+  }
+  if constexpr (T > 32) {
+    const int lane = threadIdx.x & 31;
+    const int wt = (threadIdx.x % T) >> 5;
+    __syncthreads();
+    if (lane == 0) red[token_sub * WPT + wt] = x;
+    __syncthreads();
+    float r = red[token_sub * WPT];
+#pragma unroll
+    for (int i = 1; i < WPT; ++i) r = IS_MAX ? fmaxf(r, red[token_sub * WPT + i]) : r + red[token_sub * WPT + i];
+    x = r;
+  }
+  return x;
+}
+
+template <int T, int WPT>
+HBL_DEVINL int token_reduce_i(int x, int* red, int token_sub) {
+  constexpr int W = T < 32 ? T : 32;
+#pragma unroll
+  for (int off = W / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  if constexpr (T > 32) {
+    const int lane = threadIdx.x & 31;
+    const int wt = (threadIdx.x % T) >> 5;
+    __syncthreads();
+    if (lane == 0) red[token_sub * WPT + wt] = x;
+    __syncthreads();
+    int r = 0;
+#pragma unroll
+    for (int i = 0; i < WPT; ++i) r += red[token_sub * WPT + i];
+    x = r;
+  }
+  return x;
+}
+
+// Quantise E consecutive values v[] of a token whose T threads hold the whole
+// row (K values), write codes / scale / code sum, or the fp32 values (kModeF32).
+template <int E, int T, int WPT, int MODE>
+HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool active, size_t m,
+                           float* red_f, int* red_i, int8_t* __restrict__ codes,
+                           float* __restrict__ scales, int32_t* __restrict__ csum,
+                           float* __restrict__ Xr) {
+  if constexpr (MODE == kModeF32) {
+    if (active) {
+      float4* dst = reinterpret_cast<float4*>(Xr + m * (size_t)K + (size_t)E * t);
+#pragma unroll
+      for (int q = 0; q < E / 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+    return;
+  } else {
+    float part = 0.f;
+    if constexpr (MODE == kModeInt4) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) part += fabsf(v[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < E; ++j) part = fmaxf(part, fabsf(v[j]));
+    }
+    const float r = token_reduce_f<T, WPT, MODE == kModeInt8>(part, red_f, token_sub);
+    float mult, scale;
+    int lo, hi;
+    if constexpr (MODE == kModeInt4) {
+      const float beta = __fdiv_rn(r, (float)K);               // mean |x|
+      mult = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
+      scale = __fdiv_rn(beta, kSqrt7);
+      lo = -8; hi = 7;
+    } else {
+      mult = __fdiv_rn(127.f, __fadd_rn(r, kEps));              // gamma = max |x|
+      scale = __fdiv_rn(r, 127.f);
+      lo = -128; hi = 127;
+    }
+    int cs = 0;
+    uint32_t packed[E / 4];
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) {
+      uint32_t w = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = clampi(__float2int_rn(__fmul_rn(mult, v[4 * q + i])), lo, hi);
+        cs += c;
+        w |= ((uint32_t)(c & 0xff)) << (8 * i);
+      }
+      packed[q] = w;
+    }
+    cs = token_reduce_i<T, WPT>(cs, red_i, token_sub);
+    if (active) {
+      uint4* dst = reinterpret_cast<uint4*>(codes + m * (size_t)K + (size_t)E * t);
+#pragma unroll
+      for (int q = 0; q < E / 16; ++q)
+        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      if (t == 0) {
+        scales[m] = scale;
+        if (csum) csum[m] = cs;
+      }
+    }
+  }
+}
+
+template <int LOG_K, int G, int MODE>
+__global__ void __launch_bounds__(FwhtCfg<LOG_K, G>::THREADS)
+fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ codes,
+                  float* __restrict__ scales, int32_t* __restrict__ csum, float* __restrict__ Xr) {
+  using C = FwhtCfg<LOG_K, G>;
+  constexpr int K = C::K, E = C::E, T = C::T, P = C::P;
+  extern __shared__ float smem[];
+  __shared__ float red_f[C::TPC * C::WARPS_PER_TOKEN];
+  __shared__ int red_i[C::TPC * C::WARPS_PER_TOKEN];
+
+  const int token_sub = threadIdx.x / T;
+  const int t = threadIdx.x % T;
+  const size_t m = (size_t)blockIdx.x * C::TPC + token_sub;
+  const bool active = m < (size_t)M;
+  float* sm = smem + (size_t)token_sub * K;
+
+  float v[E];
+  // Pass 0 owns the top G bits: idx = t + j*T (coalesced across threads).
+  {
+    const uint16_t* x = X + (active ? m : 0) * (size_t)K;
+#pragma unroll
+    for (int j = 0; j < E; ++j) v[j] = active ? bf16_bits_to_float(__ldg(x + t + j * T)) : 0.f;
+  }
+#pragma unroll
+  for (int p = 0; p < P; ++p) {
+    const int hi = LOG_K - p * G;
+    const int lo = hi - G > 0 ? hi - G : 0;
+    const int nb = hi - lo;        // bits processed in this pass (register bits 0..nb-1)
+    if (p > 0) {
+      // exchange: previous pass layout -> this pass layout
+      const int hi_prev = LOG_K - (p - 1) * G;
+      const int lo_prev = hi_prev - G > 0 ? hi_prev - G : 0;
+#pragma unroll
+      for (int j = 0; j < E; ++j) sm[swz<G>(pass_index<G>(t, j, lo_prev))] = v[j];
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < E; ++j) v[j] = sm[swz<G>(pass_index<G>(t, j, lo))];
+      if (p + 1 < P) __syncthreads();
+    }
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      if (r < nb) {
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+          if ((j >> r) & 1) continue;
+          const float a = v[j], b = v[j | (1 << r)];
+          v[j] = a + b;
+          v[j | (1 << r)] = a - b;
+        }
+      }
+    }
+  }
+  // Normalisation 2^(-LOG_K/2).
+  {
+    float nrm = __uint_as_float((uint32_t)(127 - LOG_K / 2) << 23);
+    if (LOG_K & 1) nrm *= 0.70710678118654752f;
+#pragma unroll
+    for (int j = 0; j < E; ++j) v[j] *= nrm;
+  }
+  quant_tail<E, T, C::WARPS_PER_TOKEN, MODE>(v, K, t, token_sub, active, m, red_f, red_i, codes,
+                                             scales, csum, Xr);
+}
+
+// Plain per-token quantiser (no Hadamard), K % 256 == 0, one token per CTA,
+// thread t holds the E consecutive values [E*t, E*t + E).
+template <int E, int MODE>
+__global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __restrict__ X, int M, int K,
+                                                          int8_t* __restrict__ codes,
+                                                          float* __restrict__ scales,
+                                                          int32_t* __restrict__ csum) {
+  __shared__ float red_f[32];
+  __shared__ int red_i[32];
+  const int t = threadIdx.x;
+  const int T = K / E;
+  const size_t m = blockIdx.x;
+  const bool active = t < T;
+  float v[E];
+  if (active) {
+    const uint4* src = reinterpret_cast<const uint4*>(X + m * (size_t)K + (size_t)E * t);
+#pragma unroll
+    for (int q = 0; q < E / 8; ++q) {
+      const uint4 u = __ldg(src + q);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+        v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < E; ++j) v[j] = 0.f;
+  }
+  // block-wide reduction over all warps (inactive threads contribute 0)
+  const int nw = blockDim.x >> 5;
+  const int lane = t & 31, wid = t >> 5;
+  float part = 0.f;
+  if (MODE == kModeInt4) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) part += fabsf(v[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < E; ++j) part = fmaxf(part, fabsf(v[j]));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, part, off);
+    part = (MODE == kModeInt4) ? part + o : fmaxf(part, o);
+  }
+  if (lane == 0) red_f[wid] = part;
+  __syncthreads();
+  float r = red_f[0];
+  for (int i = 1; i < nw; ++i) r = (MODE == kModeInt4) ? r + red_f[i] : fmaxf(r, red_f[i]);
+  float mult, scale;
+  int lo, hi;
+  if (MODE == kModeInt4) {
+    const float beta = __fdiv_rn(r, (float)K);
+    mult = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
+    scale = __fdiv_rn(beta, kSqrt7);
+    lo = -8; hi = 7;
+  } else {
+    mult = __fdiv_rn(127.f, __fadd_rn(r, kEps));
+    scale = __fdiv_rn(r, 127.f);
+    lo = -128; hi = 127;
+  }
+  int cs = 0;
+  uint32_t packed[E / 4];
+#pragma unroll
+  for (int q = 0; q < E / 4; ++q) {
+    uint32_t w = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = clampi(__float2int_rn(__fmul_rn(mult, v[4 * q + i])), lo, hi);
+      cs += active ? c : 0;
+      w |= ((uint32_t)(c & 0xff)) << (8 * i);
+    }
+    packed[q] = w;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
+  if (lane == 0) red_i[wid] = cs;
+  __syncthreads();
+  int tot = 0;
+  for (int i = 0; i < nw; ++i) tot += red_i[i];
+  if (active) {
+    if constexpr (E >= 16) {
+      uint4* dst = reinterpret_cast<uint4*>(codes + m * (size_t)K + (size_t)E * t);
+#pragma unroll
+      for (int q = 0; q < E / 16; ++q)
+        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    } else {
+      uint2* dst = reinterpret_cast<uint2*>(codes + m * (size_t)K + (size_t)E * t);
+      dst[0] = make_uint2(packed[0], packed[1]);
+    }
+    if (t == 0) {
+      scales[m] = scale;
+      if (csum) csum[m] = tot;
+    }
+  }
+}
+
+// Sum of each row of an int8 code matrix (for hbl_gemm_codes).
+__global__ void __launch_bounds__(256) code_rowsum_kernel(const int8_t* __restrict__ codes, int K,
+                                                          int32_t* __restrict__ csum) {
+  __shared__ int red[8];
+  const size_t m = blockIdx.x;
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(codes + m * (size_t)K);
+  int s = 0;
+  for (int i = threadIdx.x; i < K / 4; i += blockDim.x) {
+    const uint32_t w = __ldg(row + i);
+    s += (int)(int8_t)(w & 0xff) + (int)(int8_t)((w >> 8) & 0xff) + (int)(int8_t)((w >> 16) & 0xff) +
+         (int)(int8_t)(w >> 24);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+    csum[m] = tot;
+  }
+}
+
+}  // namespace hbl

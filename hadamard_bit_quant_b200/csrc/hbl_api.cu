@@ -1,0 +1,480 @@
+// C ABI of libhbl: argument checks, workspace layout and kernel dispatch for the
+// H-BitLinear forward (BitNet v2 architecture walkthrough, section 3.4, Eq. 9).
+// All kernels live in the headers included below (one translation unit, so the
+// device error word is shared).
+#include <mutex>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "hbl_common.cuh"
+#include "pack.cuh"
+#include "fwht_quant.cuh"
+#include "gemm_mma.cuh"
+
+namespace hbl {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  AbsSumAcc* abs_acc = nullptr;   // scratch of hbl_pack_weights
+  void* ws = nullptr;             // workspace of hbl_forward
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+// Per-kernel timing: CUDA events around each launch while enabled.
+struct Profiler {
+  struct Entry { std::string name; int launches = 0; double ms = 0.0; };
+  struct Pending { int entry; cudaEvent_t a, b; };
+  std::mutex mu;
+  bool on = false;
+  std::vector<Entry> entries;
+  std::vector<Pending> pending;
+  std::vector<cudaEvent_t> pool;
+
+  cudaEvent_t take() {
+    if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void flush() {
+    for (auto& p : pending) {
+      float ms = 0.f;
+      if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+        entries[p.entry].launches += 1;
+        entries[p.entry].ms += ms;
+      }
+      pool.push_back(p.a);
+      pool.push_back(p.b);
+    }
+    pending.clear();
+  }
+};
+Profiler g_prof;
+
+// Returns a token for prof_end (-1 when timing is off).
+int prof_begin(const char* name, cudaStream_t s) {
+  if (!g_prof.on) return -1;
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  int idx = -1;
+  for (size_t i = 0; i < g_prof.entries.size(); ++i)
+    if (g_prof.entries[i].name == name) { idx = (int)i; break; }
+  if (idx < 0) { g_prof.entries.push_back(Profiler::Entry{name, 0, 0.0}); idx = (int)g_prof.entries.size() - 1; }
+  Profiler::Pending p{idx, g_prof.take(), g_prof.take()};
+  cudaEventRecord(p.a, s);
+  g_prof.pending.push_back(p);
+  return (int)g_prof.pending.size() - 1;
+}
+
+void prof_end(int token, cudaStream_t s) {
+  if (token < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  if (token < (int)g_prof.pending.size()) cudaEventRecord(g_prof.pending[token].b, s);
+}
+
+struct ProfScope {
+  int tok;
+  cudaStream_t s;
+  ProfScope(const char* name, cudaStream_t st) : tok(prof_begin(name, st)), s(st) {}
+  ~ProfScope() { prof_end(tok, s); }
+};
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return HBL_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return HBL_ERR_UNSUPPORTED;
+  return HBL_OK;
+}
+
+// Probe the device once: sm_100 only. Also raises the dynamic shared memory
+// limit of the kernels that need more than 48 KB.
+int ensure_device(DeviceState** out) {
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.probed) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return HBL_ERR_CUDA;
+    d.supported = (prop.major == 10 && prop.minor == 0);
+    d.sm_count = prop.multiProcessorCount;
+    d.probed = true;
+    if (d.supported) {
+      cudaFuncSetAttribute(fwht_quant_kernel<13, 7, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<13, 7, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<13, 7, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<14, 7, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<14, 7, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<14, 7, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+      cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+      if (cudaGetLastError() != cudaSuccess) return HBL_ERR_CUDA;
+    }
+  }
+  if (!d.supported) return HBL_ERR_UNSUPPORTED;
+  *out = &d;
+  return HBL_OK;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+inline int ilog2(int x) { int r = 0; while ((1 << r) < x) ++r; return r; }
+inline bool misaligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+inline int launch_status() { return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA; }
+
+struct WsLayout {
+  size_t codes, scales, csum, dacc, total;
+};
+
+WsLayout ws_layout(int M, int K, int N) {
+  WsLayout L;
+  size_t off = 0;
+  L.codes = off; off = align_up(off + (size_t)M * K, 256);
+  L.scales = off; off = align_up(off + (size_t)M * 4, 256);
+  L.csum = off; off = align_up(off + (size_t)M * 4, 256);
+  L.dacc = off; off = align_up(off + (size_t)M * N * 4, 256);
+  L.total = off;
+  return L;
+}
+
+int check_weight_shape(int N, int K) {
+  if (N < 16 || N % 16 != 0) return HBL_ERR_SHAPE;
+  if (K < kKBlock || K % kKBlock != 0) return HBL_ERR_SHAPE;
+  if ((long long)N * K >= (1ll << 31)) return HBL_ERR_SHAPE;
+  return HBL_OK;
+}
+
+int check_act_shape(int M, int K, int use_hadamard) {
+  if (M < 0) return HBL_ERR_SHAPE;
+  if (use_hadamard) {
+    if (!is_pow2(K) || K < 256 || K > 32768) return HBL_ERR_SHAPE;
+  } else {
+    if (K < kKBlock || K % kKBlock != 0 || K > 65536) return HBL_ERR_SHAPE;
+  }
+  if ((long long)M * K >= (1ll << 40)) return HBL_ERR_SHAPE;
+  return HBL_OK;
+}
+
+template <int LOG_K, int G, int MODE>
+void launch_fwht(const uint16_t* X, int M, int8_t* codes, float* scales, int32_t* csum, float* Xr,
+                 cudaStream_t s) {
+  using C = FwhtCfg<LOG_K, G>;
+  const int grid = (M + C::TPC - 1) / C::TPC;
+  ProfScope ps("fwht_quant", s);
+  fwht_quant_kernel<LOG_K, G, MODE><<<grid, C::THREADS, C::SMEM, s>>>(X, M, codes, scales, csum, Xr);
+}
+
+template <int MODE>
+int dispatch_fwht(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum, float* Xr,
+                  cudaStream_t s) {
+  switch (ilog2(K)) {
+    case 8: launch_fwht<8, 4, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 9: launch_fwht<9, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 10: launch_fwht<10, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 11: launch_fwht<11, 6, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 12: launch_fwht<12, 6, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 13: launch_fwht<13, 7, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 14: launch_fwht<14, 7, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 15: launch_fwht<15, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    default: return HBL_ERR_SHAPE;
+  }
+  return launch_status();
+}
+
+template <int MODE>
+int dispatch_rows(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum,
+                  cudaStream_t s) {
+  auto blocks = [](int T) { return (T + 31) / 32 * 32; };
+  ProfScope ps("quant_rows", s);
+  if (K <= 8192) quant_rows_kernel<8, MODE><<<M, blocks(K / 8), 0, s>>>(X, M, K, codes, scales, csum);
+  else if (K <= 16384) quant_rows_kernel<16, MODE><<<M, blocks(K / 16), 0, s>>>(X, M, K, codes, scales, csum);
+  else if (K <= 32768) quant_rows_kernel<32, MODE><<<M, blocks(K / 32), 0, s>>>(X, M, K, codes, scales, csum);
+  else quant_rows_kernel<64, MODE><<<M, blocks(K / 64), 0, s>>>(X, M, K, codes, scales, csum);
+  return launch_status();
+}
+
+int run_quantize(const uint16_t* X, int M, int K, int act_bits, int use_hadamard, int8_t* codes,
+                 float* scales, int32_t* csum, cudaStream_t s) {
+  if (use_hadamard) {
+    return act_bits == 4 ? dispatch_fwht<kModeInt4>(X, M, K, codes, scales, csum, nullptr, s)
+                         : dispatch_fwht<kModeInt8>(X, M, K, codes, scales, csum, nullptr, s);
+  }
+  return act_bits == 4 ? dispatch_rows<kModeInt4>(X, M, K, codes, scales, csum, s)
+                       : dispatch_rows<kModeInt8>(X, M, K, codes, scales, csum, s);
+}
+
+// D = sum c*u over K. Chooses the token tile and a split of K so that the grid
+// covers the SMs at least twice; split partials are added atomically into a
+// zeroed D.
+int run_gemm(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, int32_t* D, int sm_count,
+             cudaStream_t s) {
+  const int nblk = K / kKBlock;
+  const int TN = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
+  const int MT = 8 * TN;
+  const int gx = (N + kMmaRowsPerCta - 1) / kMmaRowsPerCta;
+  const int gy = (M + MT - 1) / MT;
+  const long long base = (long long)gx * gy;
+  int splits = (int)((2LL * sm_count + base - 1) / base);
+  if (splits > nblk) splits = nblk;
+  if (splits < 1) splits = 1;
+  const int kps = (nblk + splits - 1) / splits;
+  splits = (nblk + kps - 1) / kps;
+  const int atomic = splits > 1;
+  if (atomic) {
+    ProfScope pm("memset_acc", s);
+    if (cudaMemsetAsync(D, 0, (size_t)M * N * 4, s) != cudaSuccess) return HBL_ERR_CUDA;
+  }
+  dim3 grid(gx, gy, splits);
+  ProfScope ps("gemm_mma", s);
+  const uint4* w = reinterpret_cast<const uint4*>(Wpk);
+  switch (TN) {
+    case 1: gemm_mma_kernel<1><<<grid, 128, 0, s>>>(codes, M, K, N, w, kps, D, atomic); break;
+    case 2: gemm_mma_kernel<2><<<grid, 128, 0, s>>>(codes, M, K, N, w, kps, D, atomic); break;
+    case 4: gemm_mma_kernel<4><<<grid, 128, 0, s>>>(codes, M, K, N, w, kps, D, atomic); break;
+    default: gemm_mma_kernel<8><<<grid, 128, 0, s>>>(codes, M, K, N, w, kps, D, atomic); break;
+  }
+  return launch_status();
+}
+
+int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
+                 int act_bits, int use_hadamard, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t s,
+                 DeviceState* d) {
+  const WsLayout L = ws_layout(M, K, N);
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return HBL_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  int8_t* codes = reinterpret_cast<int8_t*>(base + L.codes);
+  float* scales = reinterpret_cast<float*>(base + L.scales);
+  int32_t* csum = reinterpret_cast<int32_t*>(base + L.csum);
+  int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
+  int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s);
+  if (st) return st;
+  st = run_gemm(codes, M, K, N, Wpk, D, d->sm_count, s);
+  if (st) return st;
+  const long long total8 = (long long)M * N / 8;
+  ProfScope ps("dequant_store", s);
+  dequant_store_kernel<<<(unsigned)((total8 + 255) / 256), 256, 0, s>>>(D, csum, scales, wscale, M, N, Y);
+  return launch_status();
+}
+
+int check_forward_args(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
+                       int act_bits, int use_hadamard, const uint16_t* Y) {
+  if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+  if (use_hadamard != 0 && use_hadamard != 1) return HBL_ERR_INVALID_ARG;
+  int st = check_weight_shape(N, K);
+  if (st) return st;
+  st = check_act_shape(M, K, use_hadamard);
+  if (st) return st;
+  if (M > 0 && (!X || !Wpk || !wscale || !Y)) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(X) || misaligned16(Y) || misaligned16(Wpk)) return HBL_ERR_INVALID_ARG;
+  return HBL_OK;
+}
+
+}  // namespace
+}  // namespace hbl
+
+using namespace hbl;
+
+extern "C" {
+
+const char* hbl_status_string(int status) {
+  switch (status) {
+    case HBL_OK: return "HBL_OK";
+    case HBL_ERR_INVALID_ARG: return "HBL_ERR_INVALID_ARG";
+    case HBL_ERR_SHAPE: return "HBL_ERR_SHAPE";
+    case HBL_ERR_CUDA: return "HBL_ERR_CUDA";
+    case HBL_ERR_ALLOC: return "HBL_ERR_ALLOC";
+    case HBL_ERR_TIMEOUT: return "HBL_ERR_TIMEOUT";
+    case HBL_ERR_UNSUPPORTED: return "HBL_ERR_UNSUPPORTED";
+    case HBL_ERR_WORKSPACE: return "HBL_ERR_WORKSPACE";
+    default: return "HBL_ERR_UNKNOWN";
+  }
+}
+
+int hbl_version(void) { return 1; }
+
+size_t hbl_packed_bytes(int N, int K) {
+  if (N <= 0 || K <= 0) return 0;
+  return (size_t)N * (size_t)K / 4;
+}
+
+int hbl_pack_weights(const float* W, int N, int K, uint8_t* Wpk, float* wscale, hbl_stream stream) {
+  int st = check_weight_shape(N, K);
+  if (st) return st;
+  if (!W || !Wpk || !wscale) return HBL_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(Wpk) & 15u) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d->abs_acc && cudaMalloc(&d->abs_acc, sizeof(AbsSumAcc)) != cudaSuccess) {
+      d->abs_acc = nullptr;
+      return HBL_ERR_ALLOC;
+    }
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(d->abs_acc, 0, sizeof(AbsSumAcc), s) != cudaSuccess) return HBL_ERR_CUDA;
+  const long long n = (long long)N * K;
+  int blocks = d->sm_count * 4;
+  abs_sum_kernel<<<blocks, 256, 0, s>>>(W, n, d->abs_acc);
+  alpha_finalize_kernel<<<1, 32, 0, s>>>(d->abs_acc, n, wscale);
+  const long long words = n / 16;
+  ternary_pack_kernel<<<(unsigned)((words + 255) / 256), 256, 0, s>>>(W, N, K, wscale,
+                                                                      reinterpret_cast<uint32_t*>(Wpk));
+  return launch_status();
+}
+
+int hbl_unpack_weights(const uint8_t* Wpk, int N, int K, int8_t* T, hbl_stream stream) {
+  int st = check_weight_shape(N, K);
+  if (st) return st;
+  if (!Wpk || !T) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  const long long words = (long long)N * K / 16;
+  ternary_unpack_kernel<<<(unsigned)((words + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(Wpk), N, K, T);
+  return launch_status();
+}
+
+size_t hbl_workspace_bytes(int M, int K, int N) {
+  if (M < 0 || K <= 0 || N <= 0) return 0;
+  return ws_layout(M, K, N).total;
+}
+
+int hbl_forward_ws(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
+                   int act_bits, int use_hadamard, hbl_bf16* Y, void* ws, size_t ws_bytes, hbl_stream stream) {
+  int st = check_forward_args(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y);
+  if (st || M == 0) return st;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  return forward_impl(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), d);
+}
+
+int hbl_forward(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale, int act_bits,
+                int use_hadamard, hbl_bf16* Y, hbl_stream stream) {
+  int st = check_forward_args(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y);
+  if (st || M == 0) return st;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  const size_t need = ws_layout(M, K, N).total;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (d->ws_bytes < need) {
+      if (d->ws) {
+        cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+        cudaFree(d->ws);
+      }
+      d->ws = nullptr;
+      d->ws_bytes = 0;
+      if (cudaMalloc(&d->ws, need) != cudaSuccess) return HBL_ERR_ALLOC;
+      d->ws_bytes = need;
+    }
+  }
+  return forward_impl(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, d->ws, d->ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), d);
+}
+
+int hbl_hadamard_f32(const hbl_bf16* X, int M, int K, float* Xr, hbl_stream stream) {
+  int st = check_act_shape(M, K, 1);
+  if (st || M == 0) return st;
+  if (!X || !Xr) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(X) || misaligned16(Xr)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  return dispatch_fwht<kModeF32>(X, M, K, nullptr, nullptr, nullptr, Xr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard, int8_t* codes, float* scales,
+                 int32_t* csum, hbl_stream stream) {
+  if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+  if (use_hadamard != 0 && use_hadamard != 1) return HBL_ERR_INVALID_ARG;
+  int st = check_act_shape(M, K, use_hadamard);
+  if (st || M == 0) return st;
+  if (!X || !codes || !scales) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(X) || misaligned16(codes)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  return run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, int32_t* acc, hbl_stream stream) {
+  int st = check_weight_shape(N, K);
+  if (st) return st;
+  if (M < 0) return HBL_ERR_SHAPE;
+  if (M == 0) return HBL_OK;
+  if (!codes || !Wpk || !acc) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(codes) || misaligned16(Wpk) || misaligned16(acc)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // row sums go into the first M entries of a small library scratch
+  int32_t* csum = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    const size_t need = align_up((size_t)M * 4, 256);
+    if (d->ws_bytes < need) {
+      if (d->ws) { cudaStreamSynchronize(s); cudaFree(d->ws); }
+      d->ws = nullptr;
+      d->ws_bytes = 0;
+      if (cudaMalloc(&d->ws, need) != cudaSuccess) return HBL_ERR_ALLOC;
+      d->ws_bytes = need;
+    }
+    csum = static_cast<int32_t*>(d->ws);
+  }
+  code_rowsum_kernel<<<M, 256, 0, s>>>(codes, K, csum);
+  if ((st = launch_status())) return st;
+  if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
+  sub_rowsum_kernel<<<(unsigned)(((long long)M * N + 255) / 256), 256, 0, s>>>(acc, csum, M, N);
+  return launch_status();
+}
+
+int hbl_profile_enable(int enable) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.flush();
+  if (enable) g_prof.entries.clear();
+  g_prof.on = enable != 0;
+  return HBL_OK;
+}
+
+int hbl_profile_count(void) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.flush();
+  return (int)g_prof.entries.size();
+}
+
+int hbl_profile_get(int i, char* name, int name_len, int* launches, double* total_ms) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.flush();
+  if (i < 0 || i >= (int)g_prof.entries.size()) return HBL_ERR_INVALID_ARG;
+  const auto& e = g_prof.entries[i];
+  if (name && name_len > 0) {
+    std::strncpy(name, e.name.c_str(), (size_t)name_len - 1);
+    name[name_len - 1] = 0;
+  }
+  if (launches) *launches = e.launches;
+  if (total_ms) *total_ms = e.ms;
+  return HBL_OK;
+}
+
+int hbl_get_device_error(hbl_stream stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HBL_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return HBL_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return HBL_ERR_CUDA;
+  if (word & (1u << HBL_ERR_TIMEOUT)) return HBL_ERR_TIMEOUT;
+  if (word & (1u << HBL_ERR_INVALID_ARG)) return HBL_ERR_INVALID_ARG;
+  return word ? HBL_ERR_CUDA : HBL_OK;
+}
+
+}  // extern "C"

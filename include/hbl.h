@@ -1,0 +1,194 @@
+/*
+ * hbl.h -- C ABI of libhbl.so: the H-BitLinear forward of BitNet v2 on B200 (sm_100a).
+ *
+ * The operation is the one defined in "BitNet v2: Native 4-bit Activations
+ * with Hadamard Transformation for 1-bit LLMs" (architecture walkthrough,
+ * section 3.4):
+ *
+ *   Y = Q_w(W) . Q_INT8/4(X_r),   X_r = Hadamard(X)                (Eq. 9)
+ *   Q_w(W)    = alpha * RoundClip(W / (alpha + eps), -1, 1),
+ *               alpha = mean|W| over the whole tensor                (Eq. 1-2)
+ *   Hadamard(x) = H_m x, Sylvester H_m scaled by 2^(-m/2), n = 2^m    (Eq. 3-6)
+ *   Q_INT8(x) = gamma/127 * RoundClip(127/(gamma+eps) x, -128, 127),
+ *               gamma = max|x| per token                              (Eq. 7)
+ *   Q_INT4(x) = beta/sqrt7 * RoundClip(sqrt7/(beta+eps) x, -8, 7),
+ *               beta = mean|x| per token                              (Eq. 8)
+ *
+ * with eps = 1e-5 and round-half-to-even. The LN of Eq. 9 is not applied here:
+ * the layer input X is taken as already normalised.
+ *
+ * Shapes: X is M x K (tokens x in-features), W is N x K (out x in), Y is M x N;
+ * all row-major and contiguous. bf16 tensors are passed as their 16-bit
+ * patterns (hbl_bf16).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE memory owned by the caller unless stated otherwise.
+ *     The library never frees caller memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Nothing throws, aborts or prints. Arguments are checked before
+ *     any launch; a rejected call launches nothing and returns the status.
+ *   - Return value: an hbl_status (HBL_OK = 0).
+ *   - M == 0 is an empty batch: the call returns HBL_OK and launches nothing.
+ *   - Y must not overlap X; Wpk and wscale are read-only during a forward.
+ *   - Input values are expected to be finite.
+ *   - Every tensor pointer must be 16-byte aligned (HBL_ERR_INVALID_ARG otherwise).
+ */
+#ifndef HBL_H_
+#define HBL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hbl_bf16;              /* bit pattern of a bfloat16 value */
+typedef struct CUstream_st* hbl_stream; /* same type as cudaStream_t       */
+
+typedef enum {
+  HBL_OK = 0,
+  HBL_ERR_INVALID_ARG = 1, /* null pointer, act_bits not in {4,8}, bad flag          */
+  HBL_ERR_SHAPE = 2,       /* a size outside the supported set (see each call)      */
+  HBL_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed                  */
+  HBL_ERR_ALLOC = 4,       /* the library's own device allocation failed            */
+  HBL_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out                    */
+  HBL_ERR_UNSUPPORTED = 6, /* the current device is not sm_100                      */
+  HBL_ERR_WORKSPACE = 7    /* caller workspace missing or smaller than required     */
+} hbl_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hbl_status_string(int status);
+
+/* Library ABI version, currently 1. */
+int hbl_version(void);
+
+/* ------------------------------------------------------------------------
+ * Weights: ternarise and pack (offline, once per weight matrix).
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of the packed weight buffer for an N x K matrix: N*K/4 (2 bits per weight). */
+size_t hbl_packed_bytes(int N, int K);
+
+/*
+ * hbl_pack_weights -- Eq. 1-2 (section 3.4, "Weight Quantization").
+ *   W      : device fp32, N x K row-major, the latent full-precision weights.
+ *   Wpk    : device, hbl_packed_bytes(N, K) bytes, written with the ternary codes.
+ *   wscale : device, one fp32, written with alpha.
+ * alpha is the exact mean of |W| (exact sum rounded once to fp64, divided by
+ * N*K in fp64, rounded to fp32), so it does not depend on the order of
+ * summation. Codes are RoundClip(W / (alpha + eps), -1, 1) with the division
+ * in fp32.
+ * Wpk is OPAQUE: its layout is chosen for the forward kernels. Use
+ * hbl_unpack_weights for the canonical N x K view of the codes.
+ * Shapes: N >= 1, N % 16 == 0, K >= 256, K % 256 == 0, N*K < 2^31.
+ * Uses a small internal device scratch (allocated on the first call per
+ * device); calls on different streams of one device must not overlap.
+ */
+int hbl_pack_weights(const float* W, int N, int K, uint8_t* Wpk, float* wscale,
+                     hbl_stream stream);
+
+/*
+ * hbl_unpack_weights -- canonical view of packed weights.
+ *   T : device int8, N x K row-major, written with codes in {-1, 0, +1}.
+ */
+int hbl_unpack_weights(const uint8_t* Wpk, int N, int K, int8_t* T, hbl_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Forward.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of caller workspace needed by hbl_forward_ws for these sizes. */
+size_t hbl_workspace_bytes(int M, int K, int N);
+
+/*
+ * hbl_forward_ws -- H-BitLinear forward, Eq. 9 without the LN.
+ *   X            : device bf16, M x K.
+ *   Wpk, wscale  : from hbl_pack_weights for an N x K matrix.
+ *   act_bits     : 4 (Eq. 8, absmean, codes in [-8, 7]) or 8 (Eq. 7, absmax, codes in [-127, 127]).
+ *   use_hadamard : 1 = apply the Hadamard transform along K first (K must be a
+ *                  power of two, 256 <= K <= 32768); 0 = plain BitLinear
+ *                  (K % 256 == 0, K <= 65536).
+ *   Y            : device bf16, M x N, written with bf16_rne(acc * s[m] * alpha),
+ *                  acc the exact integer product of the codes, s[m] the token scale.
+ *   ws, ws_bytes : device workspace of at least hbl_workspace_bytes(M, K, N)
+ *                  bytes, 256-byte aligned; clobbered.
+ * Shapes: M >= 0, N % 16 == 0, N >= 16. Launches only kernels; makes no
+ * allocation and no synchronisation, so it may be captured in a CUDA graph.
+ */
+int hbl_forward_ws(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk,
+                   const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y,
+                   void* ws, size_t ws_bytes, hbl_stream stream);
+
+/*
+ * hbl_forward -- same as hbl_forward_ws with a library-owned workspace.
+ * The workspace is per device and grows on demand (a cudaMalloc while the
+ * stream may be busy), so this call is not for stream capture, and calls on
+ * different streams of one device must not overlap.
+ */
+int hbl_forward(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk,
+                const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y,
+                hbl_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Stage-wise entry points (the steps of the forward, for checking each one).
+ * ------------------------------------------------------------------------ */
+
+/*
+ * hbl_hadamard_f32 -- X_r = Hadamard(X) per token in fp32 (Eq. 3-5).
+ *   X  : device bf16 M x K.   Xr : device fp32 M x K.
+ * K must be a power of two, 256 <= K <= 32768.
+ */
+int hbl_hadamard_f32(const hbl_bf16* X, int M, int K, float* Xr, hbl_stream stream);
+
+/*
+ * hbl_quantize -- optional Hadamard, then the per-token quantiser (Eq. 7 / Eq. 8).
+ *   codes  : device int8 M x K.
+ *   scales : device fp32 M: gamma/127 (act_bits 8) or beta/sqrt7 (act_bits 4).
+ *   csum   : device int32 M or NULL: sum of the codes of each token.
+ */
+int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard,
+                 int8_t* codes, float* scales, int32_t* csum, hbl_stream stream);
+
+/*
+ * hbl_gemm_codes -- acc[m, n] = sum_k codes[m, k] * T[n, k], exactly, in int32.
+ *   codes : device int8 M x K (any values in [-128, 127]).
+ *   acc   : device int32 M x N.
+ * Same shape rules as hbl_forward_ws (K % 256 == 0).
+ */
+int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
+                   int32_t* acc, hbl_stream stream);
+
+/*
+ * hbl_get_device_error -- synchronises `stream`, then reads and clears the
+ * device error word that bounded waits inside the kernels set when they give
+ * up. Returns HBL_OK, HBL_ERR_TIMEOUT, or HBL_ERR_CUDA if the stream reports an
+ * error.
+ */
+int hbl_get_device_error(hbl_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Per-kernel timing of the library's own launches.
+ * While enabled, every kernel the library launches is bracketed by two CUDA
+ * events recorded on its launch stream; durations accumulate per kernel name.
+ * Meant for measurement runs, not for stream capture.
+ * ------------------------------------------------------------------------ */
+
+/* Enable (1) or disable (0) timing on the current device; enabling clears the totals. */
+int hbl_profile_enable(int enable);
+
+/* Number of distinct kernel names recorded so far (synchronises pending events). */
+int hbl_profile_count(void);
+
+/*
+ * Totals of entry i (0 <= i < hbl_profile_count()): the kernel name (copied
+ * into name, at most name_len bytes including the terminator), the number of
+ * launches and their summed device time in milliseconds.
+ */
+int hbl_profile_get(int i, char* name, int name_len, int* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HBL_H_ */

@@ -150,9 +150,9 @@ def hadamard_matrix(n: int) -> np.ndarray:
     S = np.ones((1, 1), dtype=np.float64)
     for _ in range(m):
         S = np.block([[S, S], [S, -S]])
-    H = S * (2.0 ** (-m / 2.0))
-    H.setflags(write=False)
-    return H
+    S *= 2.0 ** (-m / 2.0)
+    S.setflags(write=False)
+    return S
 
 
 def hadamard(X) -> np.ndarray:

@@ -1,0 +1,109 @@
+"""The C-ABI library: it builds, loads, exports every declared symbol, and its
+host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hadamard_bit_quant_b200 import build as hbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hbl.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    from hadamard_bit_quant_b200 import hbl
+    return hbl.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(hbl_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("hbl_pack_weights", "hbl_forward", "hbl_forward_ws", "hbl_workspace_bytes",
+                 "hbl_hadamard_f32", "hbl_quantize", "hbl_gemm_codes", "hbl_unpack_weights",
+                 "hbl_packed_bytes", "hbl_status_string", "hbl_get_device_error", "hbl_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    from hadamard_bit_quant_b200 import hbl
+    bound = {n for n, _, _ in hbl.SIGNATURES}
+    assert set(declared_functions()) <= bound
+    for n in bound:
+        assert callable(getattr(hbl, n))
+
+
+def test_host_side_queries(lib):
+    from hadamard_bit_quant_b200 import hbl
+    assert hbl.hbl_version() == 1
+    assert hbl.hbl_packed_bytes(4096, 4096) == 4096 * 4096 // 4
+    assert hbl.hbl_packed_bytes(0, 4096) == 0
+    assert hbl.hbl_status_string(0) == "HBL_OK"
+    assert hbl.hbl_status_string(2) == "HBL_ERR_SHAPE"
+    assert hbl.hbl_status_string(99) == "HBL_ERR_UNKNOWN"
+    w = hbl.hbl_workspace_bytes(16, 4096, 4096)
+    assert w >= 16 * 4096 + 16 * 4 * 2 and w % 256 == 0
+    assert hbl.hbl_workspace_bytes(0, 4096, 4096) >= 0
+
+
+BAD = 0x1000  # never dereferenced: every call below is rejected before any launch
+
+
+@pytest.mark.parametrize("args,status", [
+    # act_bits / use_hadamard
+    ((BAD, 4, 4096, 4096, BAD, BAD, 3, 1, BAD), 1),
+    ((BAD, 4, 4096, 4096, BAD, BAD, 4, 2, BAD), 1),
+    # K not a power of two with the Hadamard on, K too small, K too large
+    ((BAD, 4, 768, 4096, BAD, BAD, 4, 1, BAD), 2),
+    ((BAD, 4, 128, 4096, BAD, BAD, 4, 0, BAD), 2),
+    ((BAD, 4, 65536, 4096, BAD, BAD, 4, 1, BAD), 2),
+    # N not a multiple of 16, K not a multiple of 256
+    ((BAD, 4, 4096, 4100, BAD, BAD, 4, 1, BAD), 2),
+    ((BAD, 4, 1000, 4096, BAD, BAD, 8, 0, BAD), 2),
+    # negative M, null pointers
+    ((BAD, -1, 4096, 4096, BAD, BAD, 4, 1, BAD), 2),
+    ((None, 4, 4096, 4096, BAD, BAD, 4, 1, BAD), 1),
+    ((BAD, 4, 4096, 4096, None, BAD, 4, 1, BAD), 1),
+    ((BAD, 4, 4096, 4096, BAD, BAD, 4, 1, None), 1),
+])
+def test_forward_argument_checks(lib, args, status):
+    st = lib.hbl_forward(*args, None)
+    assert st == status
+    st = lib.hbl_forward_ws(*args, BAD, 1 << 20, None)
+    assert st == status
+
+
+def test_empty_batch_is_a_noop(lib):
+    # M == 0: nothing to do, nothing launched, HBL_OK even with null buffers
+    assert lib.hbl_forward(None, 0, 4096, 4096, None, None, 4, 1, None, None) == 0
+    assert lib.hbl_quantize(None, 0, 4096, 4, 1, None, None, None, None) == 0
+    assert lib.hbl_gemm_codes(None, 0, 4096, 4096, None, None, None) == 0
+
+
+def test_pack_argument_checks(lib):
+    assert lib.hbl_pack_weights(BAD, 4096, 1000, BAD, BAD, None) == 2
+    assert lib.hbl_pack_weights(BAD, 4095, 4096, BAD, BAD, None) == 2
+    assert lib.hbl_pack_weights(None, 4096, 4096, BAD, BAD, None) == 1
+    assert lib.hbl_pack_weights(BAD, 4096, 4096, BAD + 1, BAD, None) == 1   # Wpk not 16-byte aligned
+    assert lib.hbl_unpack_weights(BAD, 16, 100, BAD, None) == 2
+
+
+def test_quantize_and_hadamard_argument_checks(lib):
+    assert lib.hbl_quantize(BAD, 2, 4096, 5, 1, BAD, BAD, None, None) == 1
+    assert lib.hbl_quantize(BAD, 2, 3000, 4, 1, BAD, BAD, None, None) == 2
+    assert lib.hbl_hadamard_f32(BAD, 2, 3000, BAD, None) == 2
+    assert lib.hbl_hadamard_f32(None, 2, 4096, BAD, None) == 1
