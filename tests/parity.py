@@ -3,7 +3,8 @@ H-BitLinear forward).
 
 * Hadamard: per token, max |X_r,gpu - X_r,ref| <= 1e-5 * max |X_r,ref| (fp32).
 * Codes: identical except +-1 where the oracle flags a near tie, and at most
-  1e-4 of all codes may differ. Scales agree to 1e-5 relative.
+  1e-4 of all codes may differ (at least one flip allowed in cases with fewer
+  than 1e4 codes, where a rate of 1e-4 cannot be resolved). Scales agree to 1e-5 relative.
 * Integer accumulators: bit-exact given the same codes.
 * Y (bf16): |Y_gpu - Y_ref| <= 1e-2 |Y_ref| + s[m] * alpha * (differing codes
   in row m) -- the second term bounds what a tie-flipped code can change.
@@ -30,7 +31,9 @@ def check_codes(codes_gpu, codes_ref, tie_ref, scales_gpu, scales_ref):
     diff = cg != cr
     assert np.all(np.abs(cg - cr)[diff] == 1), "a code differs by more than 1"
     assert np.all(tie_ref[diff]), f"{int((diff & ~tie_ref).sum())} codes differ away from a near tie"
-    assert diff.mean() <= CODE_DIFF_FRAC, f"too many tie flips: {diff.mean():.2e}"
+    # a rate of 1e-4 cannot be resolved below 1e4 codes: small cases may flip one tie
+    allowed = max(1, int(CODE_DIFF_FRAC * diff.size))
+    assert diff.sum() <= allowed, f"too many tie flips: {int(diff.sum())} of {diff.size}"
     sg = np.asarray(scales_gpu, np.float64)
     assert np.all(np.abs(sg - scales_ref) <= SCALE_RTOL * np.abs(scales_ref) + 1e-30), "scales differ"
     return diff
