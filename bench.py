@@ -236,9 +236,8 @@ def timed_replays(torch, dist, g, warmup, steps, world):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        from hadamard_bit_quant_b200.shard import max_over_ranks
+        ms = max_over_ranks(ms, device="cuda")
         dist.barrier()
     return ms
 

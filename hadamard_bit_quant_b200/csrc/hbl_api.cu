@@ -7,10 +7,13 @@
 #include <string>
 #include <vector>
 
+#include <cuda.h>
+
 #include "hbl_common.cuh"
 #include "pack.cuh"
 #include "fwht_quant.cuh"
 #include "gemm_mma.cuh"
+#include "gemm_tc.cuh"
 
 namespace hbl {
 namespace {
@@ -117,6 +120,8 @@ int ensure_device(DeviceState** out) {
       cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
       cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
       cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+      cudaFuncSetAttribute(tc::gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
+      cudaFuncSetAttribute(tc::gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
       if (cudaGetLastError() != cudaSuccess) return HBL_ERR_CUDA;
     }
   }
@@ -245,6 +250,67 @@ int run_gemm(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, int32
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 path: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor map: rows x cols bytes, row stride `stride` bytes, box box_cols x box_rows.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
+                 uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int g_gemm_path = 0;  // 0 auto, 1 warp-level mma.sync, 2 tcgen05
+
+bool use_tc_path(int M) {
+  if (g_gemm_path == 1) return false;
+  if (g_gemm_path == 2) return true;
+  return M >= 128;
+}
+
+// bf16 output (Y != nullptr) or int32 output (acc != nullptr); D - csum either way.
+int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
+                const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
+  CUtensorMap mc, mw;
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc::kToks, true)) return HBL_ERR_CUDA;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc::kRows, false))
+    return HBL_ERR_CUDA;
+  dim3 grid((N + tc::kRows - 1) / tc::kRows, (M + tc::kToks - 1) / tc::kToks);
+  ProfScope ps("gemm_tc", s);
+  if (Y)
+    tc::gemm_tc_kernel<true><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(mc, mw, M, K, N, csum, scales, alpha, Y,
+                                                                        nullptr);
+  else
+    tc::gemm_tc_kernel<false><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(mc, mw, M, K, N, csum, nullptr, nullptr,
+                                                                         nullptr, acc);
+  return launch_status();
+}
+
 int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
                  int act_bits, int use_hadamard, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t s,
                  DeviceState* d) {
@@ -257,6 +323,7 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s);
   if (st) return st;
+  if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
   st = run_gemm(codes, M, K, N, Wpk, D, d->sm_count, s);
   if (st) return st;
   const long long total8 = (long long)M * N / 8;
@@ -432,9 +499,16 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   }
   code_rowsum_kernel<<<M, 256, 0, s>>>(codes, K, csum);
   if ((st = launch_status())) return st;
+  if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
   if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
   sub_rowsum_kernel<<<(unsigned)(((long long)M * N + 255) / 256), 256, 0, s>>>(acc, csum, M, N);
   return launch_status();
+}
+
+int hbl_set_gemm_path(int path) {
+  if (path < 0 || path > 2) return HBL_ERR_INVALID_ARG;
+  g_gemm_path = path;
+  return HBL_OK;
 }
 
 int hbl_profile_enable(int enable) {

@@ -31,6 +31,7 @@ SIGNATURES = [
     ("hbl_quantize", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _P]),
     ("hbl_gemm_codes", _I, [_P, _I, _I, _I, _P, _P, _P]),
     ("hbl_get_device_error", _I, [_P]),
+    ("hbl_set_gemm_path", _I, [_I]),
     ("hbl_profile_enable", _I, [_I]),
     ("hbl_profile_count", _I, []),
     ("hbl_profile_get", _I, [_I, ctypes.c_char_p, _I, ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double)]),
@@ -132,6 +133,10 @@ def hbl_gemm_codes(codes, M, K, N, Wpk, acc, stream=None):
 
 def hbl_get_device_error(stream=None):
     return lib().hbl_get_device_error(_stream(stream))
+
+
+def hbl_set_gemm_path(path: int) -> int:
+    return _check(lib().hbl_set_gemm_path(int(path)), "hbl_set_gemm_path")
 
 
 def hbl_profile_enable(enable: int) -> int:

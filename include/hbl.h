@@ -167,6 +167,15 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
  */
 int hbl_get_device_error(hbl_stream stream);
 
+/*
+ * hbl_set_gemm_path -- which integer-GEMM kernel the forward and
+ * hbl_gemm_codes use: 0 = by size (default: tcgen05 tensor-core kernel for
+ * M >= 128 tokens, warp-level mma.sync kernel below), 1 = always the
+ * warp-level kernel, 2 = always the tcgen05 kernel. Both give identical
+ * results; the knob exists to check and time each one. Process-wide.
+ */
+int hbl_set_gemm_path(int path);
+
 /* ------------------------------------------------------------------------
  * Per-kernel timing of the library's own launches.
  * While enabled, every kernel the library launches is bracketed by two CUDA

@@ -231,3 +231,36 @@ def test_forward_rejects_bad_workspace(L):
         L.forward(X, Wpk, wsc, 64, 4, 1, ws=small)
     assert e.value.status == 7
     assert hbl.hbl_get_device_error() == 0
+
+
+# ----------------------------------------------------------------------------- both GEMM kernels
+@pytest.fixture
+def gemm_path(L):
+    from hadamard_bit_quant_b200 import hbl
+    yield hbl.hbl_set_gemm_path
+    hbl.hbl_set_gemm_path(0)
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["mma_sync", "tcgen05"])
+@pytest.mark.parametrize("M,K,N", [(256, 256, 128), (1, 256, 16), (37, 512, 48), (300, 1024, 272),
+                                   (512, 4096, 256), (257, 2048, 130 * 16), (1024, 16384, 128)])
+def test_gemm_paths_bit_exact(L, gemm_path, path, M, K, N):
+    gemm_path(path)
+    g = torch.Generator().manual_seed(M + K + N)
+    codes = torch.randint(-128, 128, (M, K), generator=g, dtype=torch.int8)
+    W = inputs.gaussian_weights(N, K, M + 1)
+    _, T_ref = _oracle_weights(W)
+    Wpk, _ = L.pack_weights(dev(W))
+    acc = L.gemm_codes(dev(codes), Wpk, N).cpu().numpy()
+    from hadamard_bit_quant_b200 import hbl
+    assert hbl.hbl_get_device_error() == 0
+    assert np.array_equal(acc, oracle.gemm_int(codes.numpy(), T_ref))
+
+
+@pytest.mark.parametrize("path", [1, 2], ids=["mma_sync", "tcgen05"])
+def test_forward_paths(L, gemm_path, path):
+    gemm_path(path)
+    case = inputs.prefill_down_case(M=300)
+    case.K, case.N = 4096, 512
+    _forward_case(L, case.make_x(), case.make_w(), 4, 1, ws=True)
+    _forward_case(L, inputs.student_t(129, 1024, 1), inputs.gaussian_weights(80, 1024, 2), 8, 0)
