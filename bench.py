@@ -244,6 +244,7 @@ def timed_replays(torch, dist, g, warmup, steps, world):
 
 KERNEL_BYTES = {
     # algorithmic bytes per launch (what the step must move), per kernel kind
+    "gemm_decode": lambda M, K, N: N * K / 4 + M * K + 2 * M * N + 8 * M + 4,
     "gemm_mma": lambda M, K, N: N * K / 4 + M * K + 2 * M * N + 4 * M + 4,
     "fwht_quant": lambda M, K, N: M * (2 * K + K + 8),
     "quant_rows": lambda M, K, N: M * (2 * K + K + 8),
@@ -318,7 +319,7 @@ def secondary(torch, hbl, layer, inputs):
     prof = profile_kernels(torch, hbl, X, [Wpk], wsc, Y, ws, c, 3)
     ms = statistics.median(times)
     ops = 2.0 * case.M * case.N * case.K
-    gemm_ms = prof.get("gemm_mma", {}).get("ms_per_launch")
+    gemm_ms = (prof.get("gemm_tc") or prof.get("gemm_mma") or {}).get("ms_per_launch")
     out["prefill M=4096 K=16384 N=4096 a4"] = {
         "ms_forward": ms, "tokens_per_s": case.M / (ms * 1e-3), "TOPS": ops / (ms * 1e-3) / 1e12,
         "gemm_ms": gemm_ms, "gemm_TOPS": (ops / (gemm_ms * 1e-3) / 1e12) if gemm_ms else None,
@@ -404,6 +405,29 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def profile_case(which: str):
+    """A short, fixed run for ncu captures: pack once, then two forwards of one config."""
+    import torch
+    from hadamard_bit_quant_b200 import hbl, inputs, layer
+    torch.cuda.set_device(0)
+    hbl.lib()
+    if which == "prefill":
+        case = inputs.prefill_down_case()
+    elif which == "decode":
+        case = [c for c in inputs.decode_oproj_cases((HEAD["M"],), (HEAD["act_bits"],))][0]
+    else:
+        raise SystemExit(f"unknown profile case {which}")
+    X = case.make_x().cuda()
+    Wpk, wsc = layer.pack_weights(case.make_w().cuda())
+    ws = layer.workspace(case.M, case.K, case.N, "cuda")
+    for _ in range(2):
+        Y = layer.forward(X, Wpk, wsc, case.N, case.act_bits, case.use_hadamard, ws=ws)
+    torch.cuda.synchronize()
+    assert hbl.hbl_get_device_error() == 0
+    print(f"profile case {which}: {case.label} ok, |Y|max={Y.float().abs().max().item():.3f}")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -412,7 +436,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile-case", choices=["prefill", "decode"], default=None,
+                    help="run one short fixed case (for ncu captures) and exit")
     args = ap.parse_args()
+    if args.profile_case:
+        return profile_case(args.profile_case)
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = dist_env()

@@ -140,13 +140,49 @@ HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool acti
     }
     cs = token_reduce_i<T, WPT>(cs, red_i, token_sub);
     if (active) {
-      uint4* dst = reinterpret_cast<uint4*>(codes + m * (size_t)K + (size_t)E * t);
+      if constexpr (E >= 16) {
+        uint4* dst = reinterpret_cast<uint4*>(codes + m * (size_t)K + (size_t)E * t);
 #pragma unroll
-      for (int q = 0; q < E / 16; ++q)
-        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        for (int q = 0; q < E / 16; ++q)
+          dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      } else {
+        *reinterpret_cast<uint2*>(codes + m * (size_t)K + (size_t)E * t) = make_uint2(packed[0], packed[1]);
+      }
       if (t == 0) {
         scales[m] = scale;
         if (csum) csum[m] = cs;
+      }
+    }
+  }
+}
+
+// Butterflies over register-index bits 0..nb-1 of v[0..E). Bit 0 pairs the two
+// halves of a register pair (scalar adds); every higher bit pairs whole
+// register pairs, done with the packed two-lane fp32 add of sm_100 -- the
+// same IEEE additions, half the instructions.
+template <int E>
+HBL_DEVINL void butterflies(float (&v)[E], int nb) {
+  if (nb > 0) {
+#pragma unroll
+    for (int j = 0; j < E; j += 2) {
+      const float a = v[j], b = v[j + 1];
+      v[j] = a + b;
+      v[j + 1] = a - b;
+    }
+  }
+#pragma unroll
+  for (int r = 1; r < 8; ++r) {
+    if (r < nb && (1 << r) < E) {
+#pragma unroll
+      for (int j = 0; j < E; j += 2) {
+        if ((j >> r) & 1) continue;
+        const int k = j | (1 << r);
+        const float2 a = make_float2(v[j], v[j + 1]);
+        const float2 b = make_float2(v[k], v[k + 1]);
+        const float2 s = __fadd2_rn(a, b);
+        const float2 d = __fadd2_rn(a, make_float2(-b.x, -b.y));
+        v[j] = s.x; v[j + 1] = s.y;
+        v[k] = d.x; v[k + 1] = d.y;
       }
     }
   }
@@ -168,6 +204,11 @@ fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ co
   const bool active = m < (size_t)M;
   float* sm = smem + (size_t)token_sub * K;
 
+  // Programmatic dependent launch: let the consumer grid launch now (it only
+  // prefetches weights until this grid completes), and wait for the producer
+  // of X before reading it. Both are no-ops without the launch attribute.
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   float v[E];
   // Pass 0 owns the top G bits: idx = t + j*T (coalesced across threads).
   {
@@ -191,25 +232,19 @@ fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ co
       for (int j = 0; j < E; ++j) v[j] = sm[swz<G>(pass_index<G>(t, j, lo))];
       if (p + 1 < P) __syncthreads();
     }
-#pragma unroll
-    for (int r = 0; r < G; ++r) {
-      if (r < nb) {
-#pragma unroll
-        for (int j = 0; j < E; ++j) {
-          if ((j >> r) & 1) continue;
-          const float a = v[j], b = v[j | (1 << r)];
-          v[j] = a + b;
-          v[j | (1 << r)] = a - b;
-        }
-      }
-    }
+    butterflies<E>(v, nb);
   }
   // Normalisation 2^(-LOG_K/2).
   {
     float nrm = __uint_as_float((uint32_t)(127 - LOG_K / 2) << 23);
     if (LOG_K & 1) nrm *= 0.70710678118654752f;
+    const float2 n2 = make_float2(nrm, nrm);
 #pragma unroll
-    for (int j = 0; j < E; ++j) v[j] *= nrm;
+    for (int j = 0; j < E; j += 2) {
+      const float2 r = __fmul2_rn(make_float2(v[j], v[j + 1]), n2);
+      v[j] = r.x;
+      v[j + 1] = r.y;
+    }
   }
   quant_tail<E, T, C::WARPS_PER_TOKEN, MODE>(v, K, t, token_sub, active, m, red_f, red_i, codes,
                                              scales, csum, Xr);
@@ -228,6 +263,8 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
   const int T = K / E;
   const size_t m = blockIdx.x;
   const bool active = t < T;
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   float v[E];
   if (active) {
     const uint4* src = reinterpret_cast<const uint4*>(X + m * (size_t)K + (size_t)E * t);

@@ -14,6 +14,7 @@
 #include "fwht_quant.cuh"
 #include "gemm_mma.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_decode.cuh"
 
 namespace hbl {
 namespace {
@@ -120,6 +121,17 @@ int ensure_device(DeviceState** out) {
       cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
       cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
       cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+      {
+        const int mx = 200 * 1024;
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+        cudaFuncSetAttribute(dec::gemm_decode_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+      }
       cudaFuncSetAttribute(tc::gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
       cudaFuncSetAttribute(tc::gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
       if (cudaGetLastError() != cudaSuccess) return HBL_ERR_CUDA;
@@ -169,18 +181,56 @@ int check_act_shape(int M, int K, int use_hadamard) {
   return HBL_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream drains; it must execute griddepcontrol.wait
+// before touching anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 template <int LOG_K, int G, int MODE>
 void launch_fwht(const uint16_t* X, int M, int8_t* codes, float* scales, int32_t* csum, float* Xr,
                  cudaStream_t s) {
   using C = FwhtCfg<LOG_K, G>;
   const int grid = (M + C::TPC - 1) / C::TPC;
   ProfScope ps("fwht_quant", s);
-  fwht_quant_kernel<LOG_K, G, MODE><<<grid, C::THREADS, C::SMEM, s>>>(X, M, codes, scales, csum, Xr);
+  launch_pdl(fwht_quant_kernel<LOG_K, G, MODE>, dim3(grid), dim3(C::THREADS), C::SMEM, s, X, M, codes, scales,
+             csum, Xr);
 }
+
+// Few tokens: more threads per token (8 or 16 values each) for latency.
+template <int MODE>
+bool dispatch_fwht_latency(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum,
+                           float* Xr, cudaStream_t s) {
+  switch (ilog2(K)) {
+    case 10: launch_fwht<10, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
+    case 11: launch_fwht<11, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
+    case 12: launch_fwht<12, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
+    case 13: launch_fwht<13, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
+    case 14: launch_fwht<14, 4, MODE>(X, M, codes, scales, csum, Xr, s); return true;
+    default: return false;
+  }
+}
+
+constexpr int kLatencyTokens = 64;
 
 template <int MODE>
 int dispatch_fwht(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum, float* Xr,
                   cudaStream_t s) {
+  if (M <= kLatencyTokens && dispatch_fwht_latency<MODE>(X, M, K, codes, scales, csum, Xr, s))
+    return launch_status();
   switch (ilog2(K)) {
     case 8: launch_fwht<8, 4, MODE>(X, M, codes, scales, csum, Xr, s); break;
     case 9: launch_fwht<9, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
@@ -200,10 +250,14 @@ int dispatch_rows(const uint16_t* X, int M, int K, int8_t* codes, float* scales,
                   cudaStream_t s) {
   auto blocks = [](int T) { return (T + 31) / 32 * 32; };
   ProfScope ps("quant_rows", s);
-  if (K <= 8192) quant_rows_kernel<8, MODE><<<M, blocks(K / 8), 0, s>>>(X, M, K, codes, scales, csum);
-  else if (K <= 16384) quant_rows_kernel<16, MODE><<<M, blocks(K / 16), 0, s>>>(X, M, K, codes, scales, csum);
-  else if (K <= 32768) quant_rows_kernel<32, MODE><<<M, blocks(K / 32), 0, s>>>(X, M, K, codes, scales, csum);
-  else quant_rows_kernel<64, MODE><<<M, blocks(K / 64), 0, s>>>(X, M, K, codes, scales, csum);
+  if (K <= 8192)
+    launch_pdl(quant_rows_kernel<8, MODE>, dim3(M), dim3(blocks(K / 8)), 0, s, X, M, K, codes, scales, csum);
+  else if (K <= 16384)
+    launch_pdl(quant_rows_kernel<16, MODE>, dim3(M), dim3(blocks(K / 16)), 0, s, X, M, K, codes, scales, csum);
+  else if (K <= 32768)
+    launch_pdl(quant_rows_kernel<32, MODE>, dim3(M), dim3(blocks(K / 32)), 0, s, X, M, K, codes, scales, csum);
+  else
+    launch_pdl(quant_rows_kernel<64, MODE>, dim3(M), dim3(blocks(K / 64)), 0, s, X, M, K, codes, scales, csum);
   return launch_status();
 }
 
@@ -311,6 +365,32 @@ int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, co
   return launch_status();
 }
 
+bool decode_path_fits(int M, int K) {
+  return M <= kLatencyTokens && dec::smem_bytes(K, 8) <= 200 * 1024;
+}
+
+int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
+                    const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
+  const int TN = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
+  const dim3 grid((N + dec::kRows - 1) / dec::kRows);
+  const size_t smem = dec::smem_bytes(K, TN);
+  ProfScope ps("gemm_decode", s);
+  cudaError_t e;
+#define HBL_DEC(TN_)                                                                                           \
+  e = Y ? launch_pdl(dec::gemm_decode_kernel<TN_, true>, grid, dim3(dec::kThreads), smem, s, codes, csum, scales, \
+                     alpha, M, K, N, Wpk, Y, (int32_t*)nullptr)                                                 \
+        : launch_pdl(dec::gemm_decode_kernel<TN_, false>, grid, dim3(dec::kThreads), smem, s, codes, csum,       \
+                     (const float*)nullptr, (const float*)nullptr, M, K, N, Wpk, (uint16_t*)nullptr, acc)
+  switch (TN) {
+    case 1: HBL_DEC(1); break;
+    case 2: HBL_DEC(2); break;
+    case 4: HBL_DEC(4); break;
+    default: HBL_DEC(8); break;
+  }
+#undef HBL_DEC
+  return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
+}
+
 int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
                  int act_bits, int use_hadamard, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t s,
                  DeviceState* d) {
@@ -324,6 +404,8 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s);
   if (st) return st;
   if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
+  if (g_gemm_path != 1 && decode_path_fits(M, K))
+    return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
   st = run_gemm(codes, M, K, N, Wpk, D, d->sm_count, s);
   if (st) return st;
   const long long total8 = (long long)M * N / 8;
@@ -500,6 +582,8 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   code_rowsum_kernel<<<M, 256, 0, s>>>(codes, K, csum);
   if ((st = launch_status())) return st;
   if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
+  if (g_gemm_path != 1 && decode_path_fits(M, K))
+    return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
   if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
   sub_rowsum_kernel<<<(unsigned)(((long long)M * N + 255) / 256), 256, 0, s>>>(acc, csum, M, N);
   return launch_status();

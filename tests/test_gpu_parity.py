@@ -241,8 +241,8 @@ def gemm_path(L):
     hbl.hbl_set_gemm_path(0)
 
 
-@pytest.mark.parametrize("path", [1, 2], ids=["mma_sync", "tcgen05"])
-@pytest.mark.parametrize("M,K,N", [(256, 256, 128), (1, 256, 16), (37, 512, 48), (300, 1024, 272),
+@pytest.mark.parametrize("path", [0, 1, 2], ids=["auto", "mma_sync", "tcgen05"])
+@pytest.mark.parametrize("M,K,N", [(256, 256, 128), (16, 4096, 512), (64, 32768, 32), (33, 1024, 144), (1, 256, 16), (37, 512, 48), (300, 1024, 272),
                                    (512, 4096, 256), (257, 2048, 130 * 16), (1024, 16384, 128)])
 def test_gemm_paths_bit_exact(L, gemm_path, path, M, K, N):
     gemm_path(path)
@@ -264,3 +264,37 @@ def test_forward_paths(L, gemm_path, path):
     case.K, case.N = 4096, 512
     _forward_case(L, case.make_x(), case.make_w(), 4, 1, ws=True)
     _forward_case(L, inputs.student_t(129, 1024, 1), inputs.gaussian_weights(80, 1024, 2), 8, 0)
+
+
+def test_chained_forwards_match_synchronised(L):
+    """Back-to-back forwards on one stream, each consuming the previous output
+    (programmatic dependent launches overlap their prologues), must give the
+    same bits as the same chain with a device synchronisation after each step,
+    and as the chain replayed from a CUDA graph."""
+    K = N = 4096
+    layers = [L.pack_weights(dev(inputs.gaussian_weights(N, K, 50 + i))) for i in range(6)]
+    for M, a in ((16, 4), (3, 8), (200, 4)):
+        X0 = dev(inputs.gaussian_with_outliers(M, K, 9, [5, 700], 30.0))
+        ws = L.workspace(M, K, N, "cuda")
+
+        def chain(sync):
+            x = X0
+            for Wpk, wsc in layers:
+                x = L.forward(x, Wpk, wsc, N, a, 1, ws=ws)
+                if sync:
+                    torch.cuda.synchronize()
+            return x
+
+        ref = chain(True).clone()
+        got = chain(False).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(ref, got)
+        outs = []
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            outs.append(chain(False))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(ref, outs[0])
+        from hadamard_bit_quant_b200 import hbl
+        assert hbl.hbl_get_device_error() == 0
