@@ -200,11 +200,27 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// Raise a kernel's dynamic shared memory limit once per device (needed above 48 KB).
+template <typename F>
+void ensure_smem_attr(F* func, size_t bytes) {
+  if (bytes <= 48 * 1024) return;
+  static std::mutex mu;
+  static std::vector<std::pair<int, const void*>> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  for (auto& e : done)
+    if (e.first == dev && e.second == (const void*)func) return;
+  cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  done.emplace_back(dev, (const void*)func);
+}
+
 template <int LOG_K, int G, int MODE>
 void launch_fwht(const uint16_t* X, int M, int8_t* codes, float* scales, int32_t* csum, float* Xr,
                  cudaStream_t s) {
   using C = FwhtCfg<LOG_K, G>;
   const int grid = (M + C::TPC - 1) / C::TPC;
+  ensure_smem_attr(fwht_quant_kernel<LOG_K, G, MODE>, C::SMEM);
   ProfScope ps("fwht_quant", s);
   launch_pdl(fwht_quant_kernel<LOG_K, G, MODE>, dim3(grid), dim3(C::THREADS), C::SMEM, s, X, M, codes, scales,
              csum, Xr);
@@ -636,3 +652,4 @@ int hbl_get_device_error(hbl_stream stream) {
 }
 
 }  // extern "C"
+
