@@ -276,3 +276,83 @@ def forward_rows(X, T, alpha, act_bits: int, use_hadamard: int, rows, cols=None)
     if cols is not None:
         T = T[np.asarray(cols)]
     return forward(X, T, alpha, act_bits, use_hadamard)
+
+
+# ---------------------------------------------------------------------------
+# Beyond the forward of Eq. 9 without LN: the LN prologue, the
+# weight-and-activation rotation variant, the Hadamard backward and the
+# post-RoPE QKV quantiser.
+# ---------------------------------------------------------------------------
+RMS_EPS = 1e-5   # reading: the pages give no epsilon for the RMSNorm; the quantisers' 1e-5 is reused
+
+
+def rmsnorm(X, gain=None):
+    """LN of Eq. 9, "RMS normalization in practice" (section 3.4, "H-BitLinear:
+    The Composite Layer"): x / sqrt(mean(x^2) + eps), times an optional
+    per-channel gain. fp64."""
+    X = np.asarray(X, dtype=np.float64)
+    r = 1.0 / np.sqrt(np.mean(X * X, axis=1) + RMS_EPS)
+    Y = X * r[:, None]
+    if gain is not None:
+        Y = Y * np.asarray(gain, dtype=np.float64)[None, :]
+    return Y
+
+
+def forward_ln(X, gain, T, alpha, act_bits: int, use_hadamard: int) -> dict:
+    """H-BitLinear with its LN: X_r = Hadamard(LN(X)), Y = Q_w(W) . Q(X_r)  [Eq. 9]."""
+    return forward(rmsnorm(X, gain), T, alpha, act_bits, use_hadamard)
+
+
+def rotate_weights(W) -> np.ndarray:
+    """W H^T of the weight-and-activation rotation variant (section 3.4, ablation
+    of Table 5): every weight row w becomes H w. Returned as fp32 (the precision
+    the ternary decision is taken in)."""
+    W = np.asarray(W, dtype=np.float64)
+    H = hadamard_matrix(W.shape[1])
+    return (W @ H.T).astype(np.float32)
+
+
+def rotated_weight_quant(W):
+    """Q_w(W H^T): alpha and ternary codes of the rotated weights  [Eq. 1 on W H^T]."""
+    return weight_quant(rotate_weights(W))
+
+
+def hadamard_backward(G) -> np.ndarray:
+    """dL/dX = H^T dL/dX_r for every token (row) of G  [section 3.4, Eq. 10].
+
+    Written with the transpose, as in the chain rule; H is symmetric, so this
+    equals another forward transform. fp64.
+    """
+    G = np.asarray(G, dtype=np.float64)
+    H = hadamard_matrix(G.shape[1])
+    return G @ H           # row form of H^T g
+
+
+def quantize_qkv(Xh, bits: int, bos_rows=()):
+    """Post-RoPE QKV quantiser (section 3.4, "QKV Attention Quantization"):
+    unsigned integers from the absmax of each head vector.
+
+    Reading: gamma = max|x| over one head of one token; the interval
+    [-gamma, gamma] maps onto [0, 2^b - 1]:
+        u = RoundClip((2^b - 1)/2 * (x / (gamma + eps) + 1), 0, 2^b - 1),
+    dequantised as (2u / (2^b - 1) - 1) * gamma. Rows listed in bos_rows (the
+    BOS token's heads) use 8 bits whatever `bits` is.
+    Xh: (rows, d) head vectors. Returns (codes uint8, gamma fp64, bits per row,
+    near-tie map).
+    """
+    Xh = np.asarray(Xh, dtype=np.float64)
+    b = np.full(Xh.shape[0], int(bits))
+    b[list(bos_rows)] = 8
+    top = (2.0 ** b - 1.0)[:, None]
+    gamma = np.max(np.abs(Xh), axis=1)
+    v = 0.5 * top * (Xh / (gamma + EPS)[:, None] + 1.0)
+    u = np.minimum(np.maximum(np.rint(v), 0.0), top)
+    f = np.floor(v)
+    near = np.abs((v - f) - 0.5) < TIE_WINDOW
+    differ = np.minimum(np.maximum(f, 0.0), top) != np.minimum(np.maximum(f + 1.0, 0.0), top)
+    return u.astype(np.uint8), gamma, b, near & differ
+
+
+def dequantize_qkv(u, gamma, b):
+    top = (2.0 ** np.asarray(b, dtype=np.float64) - 1.0)[:, None]
+    return (2.0 * np.asarray(u, dtype=np.float64) / top - 1.0) * np.asarray(gamma, np.float64)[:, None]
