@@ -653,3 +653,50 @@ int hbl_get_device_error(hbl_stream stream) {
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the workspace lives in a fixed device array that
+// is part of the library image, so this entry point never allocates.
+// ---------------------------------------------------------------------------
+namespace hbl {
+namespace {
+
+constexpr size_t kNoAllocBytes = (size_t)8 << 20;  // 8 MiB, held on every device that loads the library
+
+static __device__ __align__(256) unsigned char g_noalloc_ws[kNoAllocBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_ws on the current device. The host-side name of
+// the array is not a device address; it is looked up once per device, with
+// that device current, and cached.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  int st = current_device(&dev);
+  if (st) return st;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || p == nullptr) return HBL_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HBL_OK;
+}
+
+}  // namespace
+}  // namespace hbl
+
+extern "C" int hbl_forward_noalloc(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk,
+                                   const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y,
+                                   hbl_stream stream) {
+  int st = check_forward_args(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y);
+  if (st || M == 0) return st;
+  if (ws_layout(M, K, N).total > kNoAllocBytes) return HBL_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  void* ws = nullptr;
+  if ((st = noalloc_scratch(&ws))) return st;
+  return forward_impl(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, ws, kNoAllocBytes,
+                      reinterpret_cast<cudaStream_t>(stream), d);
+}

@@ -27,6 +27,7 @@ SIGNATURES = [
     ("hbl_workspace_bytes", _Z, [_I, _I, _I]),
     ("hbl_forward_ws", _I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P, _Z, _P]),
     ("hbl_forward", _I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P]),
+    ("hbl_forward_noalloc", _I, [_P, _I, _I, _I, _P, _P, _I, _I, _P, _P]),
     ("hbl_hadamard_f32", _I, [_P, _I, _I, _P, _P]),
     ("hbl_quantize", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _P]),
     ("hbl_gemm_codes", _I, [_P, _I, _I, _I, _P, _P, _P]),
@@ -115,6 +116,12 @@ def hbl_forward_ws(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, ws, ws_by
 def hbl_forward(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, stream=None):
     return _check(lib().hbl_forward(_ptr(X), M, K, N, _ptr(Wpk), _ptr(wscale), act_bits, use_hadamard,
                                     _ptr(Y), _stream(stream)), "hbl_forward")
+
+
+def hbl_forward_noalloc(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, stream=None):
+    """Forward with the library's fixed 8 MiB device workspace: no allocation (see include/hbl.h)."""
+    return _check(lib().hbl_forward_noalloc(_ptr(X), M, K, N, _ptr(Wpk), _ptr(wscale), act_bits, use_hadamard,
+                                            _ptr(Y), _stream(stream)), "hbl_forward_noalloc")
 
 
 def hbl_hadamard_f32(X, M, K, Xr, stream=None):

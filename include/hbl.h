@@ -130,6 +130,33 @@ int hbl_forward(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk,
                 const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y,
                 hbl_stream stream);
 
+/*
+ * hbl_forward_noalloc -- the same forward as hbl_forward_ws, for callers that
+ * cannot allocate device memory: for example a serving process whose memory
+ * pool has already reserved nearly all of HBM (a cudaMalloc would fail), code
+ * that must not pay the device-wide synchronisation a cudaMalloc/cudaFree can
+ * imply, or a host framework that forbids its plugins from allocating.
+ * The paper has no counterpart; this is a deployment convenience.
+ *
+ * The workspace is a fixed 8 MiB device array inside the library image,
+ * reserved on every GPU that loads the library until the process exits. The
+ * call makes no cudaMalloc/cudaFree and no other allocation.
+ *   - Sizes whose workspace, hbl_workspace_bytes(M, K, N), exceeds 8 MiB are
+ *     rejected with HBL_ERR_WORKSPACE before any launch (use hbl_forward_ws
+ *     with your own buffer for those, e.g. large prefill batches).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; whatever must start at zero is cleared by the call itself.
+ *     Calls whose execution overlaps on the GPU (different streams, or
+ *     different host threads) race on the array: serialise them.
+ * Arguments, shapes and results are those of hbl_forward_ws.
+ */
+int hbl_forward_noalloc(const hbl_bf16* X, int M, int K, int N, const uint8_t* Wpk,
+                        const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y,
+                        hbl_stream stream);
+
 /* ------------------------------------------------------------------------
  * Stage-wise entry points (the steps of the forward, for checking each one).
  * ------------------------------------------------------------------------ */
