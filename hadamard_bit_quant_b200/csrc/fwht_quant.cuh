@@ -138,7 +138,7 @@ HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool acti
       }
       packed[q] = w;
     }
-    cs = token_reduce_i<T, WPT>(cs, red_i, token_sub);
+    if (csum != nullptr) cs = token_reduce_i<T, WPT>(cs, red_i, token_sub);   // uniform branch
     if (active) {
       if constexpr (E >= 16) {
         uint4* dst = reinterpret_cast<uint4*>(codes + m * (size_t)K + (size_t)E * t);
@@ -188,9 +188,17 @@ HBL_DEVINL void butterflies(float (&v)[E], int nb) {
   }
 }
 
-template <int LOG_K, int G, int MODE>
+// RMSNorm epsilon of the LN prologue (a reading: the pages give none; the
+// quantisers' 1e-5 is reused).
+constexpr float kRmsEps = 1e-5f;
+
+// IN_F32: X is fp32 (gradients, latent weights) instead of bf16.
+// LN: apply the RMSNorm of Eq. 9 first: x * gain / sqrt(mean(x^2) + eps). The
+// per-channel gain is applied on load; the per-token factor commutes with the
+// transform and is folded into the final normalisation.
+template <int LOG_K, int G, int MODE, bool IN_F32 = false, bool LN = false>
 __global__ void __launch_bounds__(FwhtCfg<LOG_K, G>::THREADS)
-fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ codes,
+fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ gain, int8_t* __restrict__ codes,
                   float* __restrict__ scales, int32_t* __restrict__ csum, float* __restrict__ Xr) {
   using C = FwhtCfg<LOG_K, G>;
   constexpr int K = C::K, E = C::E, T = C::T, P = C::P;
@@ -210,11 +218,23 @@ fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ co
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
   float v[E];
+  float ssq = 0.f;
   // Pass 0 owns the top G bits: idx = t + j*T (coalesced across threads).
   {
-    const uint16_t* x = X + (active ? m : 0) * (size_t)K;
+    const size_t row = (active ? m : 0) * (size_t)K;
 #pragma unroll
-    for (int j = 0; j < E; ++j) v[j] = active ? bf16_bits_to_float(__ldg(x + t + j * T)) : 0.f;
+    for (int j = 0; j < E; ++j) {
+      float x = 0.f;
+      if (active) {
+        if constexpr (IN_F32) x = __ldg(reinterpret_cast<const float*>(Xv) + row + t + j * T);
+        else x = bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(Xv) + row + t + j * T));
+      }
+      if constexpr (LN) {
+        ssq = __fmaf_rn(x, x, ssq);
+        if (gain) x = __fmul_rn(x, __ldg(gain + t + j * T));
+      }
+      v[j] = x;
+    }
   }
 #pragma unroll
   for (int p = 0; p < P; ++p) {
@@ -234,10 +254,15 @@ fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ co
     }
     butterflies<E>(v, nb);
   }
-  // Normalisation 2^(-LOG_K/2).
+  // Normalisation 2^(-LOG_K/2) (times the RMSNorm factor with LN).
   {
     float nrm = __uint_as_float((uint32_t)(127 - LOG_K / 2) << 23);
     if (LOG_K & 1) nrm *= 0.70710678118654752f;
+    if constexpr (LN) {
+      const float tot = token_reduce_f<T, C::WARPS_PER_TOKEN, false>(ssq, red_f, token_sub);
+      const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)K), kRmsEps)));
+      nrm = __fmul_rn(nrm, r);
+    }
     const float2 n2 = make_float2(nrm, nrm);
 #pragma unroll
     for (int j = 0; j < E; j += 2) {
@@ -252,8 +277,9 @@ fwht_quant_kernel(const uint16_t* __restrict__ X, int M, int8_t* __restrict__ co
 
 // Plain per-token quantiser (no Hadamard), K % 256 == 0, one token per CTA,
 // thread t holds the E consecutive values [E*t, E*t + E).
-template <int E, int MODE>
+template <int E, int MODE, bool LN = false>
 __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __restrict__ X, int M, int K,
+                                                          const float* __restrict__ gain,
                                                           int8_t* __restrict__ codes,
                                                           float* __restrict__ scales,
                                                           int32_t* __restrict__ csum) {
@@ -285,6 +311,24 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
   // block-wide reduction over all warps (inactive threads contribute 0)
   const int nw = blockDim.x >> 5;
   const int lane = t & 31, wid = t >> 5;
+  if constexpr (LN) {
+    float q = 0.f;
+#pragma unroll
+    for (int j = 0; j < E; ++j) q = __fmaf_rn(v[j], v[j], q);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+    if (lane == 0) red_f[wid] = q;
+    __syncthreads();
+    float tot = 0.f;
+    for (int i = 0; i < nw; ++i) tot += red_f[i];
+    __syncthreads();
+    const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)K), kRmsEps)));
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const float gj = (gain && active) ? __ldg(gain + E * t + j) : 1.f;
+      v[j] = __fmul_rn(__fmul_rn(v[j], gj), r);
+    }
+  }
   float part = 0.f;
   if (MODE == kModeInt4) {
 #pragma unroll

@@ -15,6 +15,7 @@
 #include "gemm_mma.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_decode.cuh"
+#include "qkv_quant.cuh"
 
 namespace hbl {
 namespace {
@@ -112,15 +113,6 @@ int ensure_device(DeviceState** out) {
     d.sm_count = prop.multiProcessorCount;
     d.probed = true;
     if (d.supported) {
-      cudaFuncSetAttribute(fwht_quant_kernel<13, 7, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<13, 7, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<13, 7, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<14, 7, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<14, 7, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<14, 7, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
-      cudaFuncSetAttribute(fwht_quant_kernel<15, 5, kModeF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
       {
         const int mx = 200 * 1024;
         cudaFuncSetAttribute(dec::gemm_decode_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
@@ -215,76 +207,92 @@ void ensure_smem_attr(F* func, size_t bytes) {
   done.emplace_back(dev, (const void*)func);
 }
 
-template <int LOG_K, int G, int MODE>
-void launch_fwht(const uint16_t* X, int M, int8_t* codes, float* scales, int32_t* csum, float* Xr,
-                 cudaStream_t s) {
-  using C = FwhtCfg<LOG_K, G>;
-  const int grid = (M + C::TPC - 1) / C::TPC;
-  ensure_smem_attr(fwht_quant_kernel<LOG_K, G, MODE>, C::SMEM);
-  ProfScope ps("fwht_quant", s);
-  launch_pdl(fwht_quant_kernel<LOG_K, G, MODE>, dim3(grid), dim3(C::THREADS), C::SMEM, s, X, M, codes, scales,
-             csum, Xr);
-}
+// Arguments of one Hadamard(+quantise) launch.
+struct FwhtArgs {
+  const void* X;        // bf16 or fp32 rows
+  int M;
+  const float* gain;    // RMSNorm gain (LN only), may be null
+  int8_t* codes;
+  float* scales;
+  int32_t* csum;
+  float* Xr;            // fp32 output (kModeF32)
+};
 
-// Few tokens: more threads per token (8 or 16 values each) for latency.
-template <int MODE>
-bool dispatch_fwht_latency(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum,
-                           float* Xr, cudaStream_t s) {
-  switch (ilog2(K)) {
-    case 10: launch_fwht<10, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
-    case 11: launch_fwht<11, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
-    case 12: launch_fwht<12, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
-    case 13: launch_fwht<13, 3, MODE>(X, M, codes, scales, csum, Xr, s); return true;
-    case 14: launch_fwht<14, 4, MODE>(X, M, codes, scales, csum, Xr, s); return true;
-    default: return false;
-  }
+template <int LOG_K, int G, int MODE, bool IN_F32, bool LN>
+void launch_fwht(const FwhtArgs& a, cudaStream_t s) {
+  using C = FwhtCfg<LOG_K, G>;
+  const int grid = (a.M + C::TPC - 1) / C::TPC;
+  ensure_smem_attr(fwht_quant_kernel<LOG_K, G, MODE, IN_F32, LN>, C::SMEM);
+  ProfScope ps("fwht_quant", s);
+  launch_pdl(fwht_quant_kernel<LOG_K, G, MODE, IN_F32, LN>, dim3(grid), dim3(C::THREADS), C::SMEM, s, a.X, a.M,
+             a.gain, a.codes, a.scales, a.csum, a.Xr);
 }
 
 constexpr int kLatencyTokens = 64;
 
-template <int MODE>
-int dispatch_fwht(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum, float* Xr,
-                  cudaStream_t s) {
-  if (M <= kLatencyTokens && dispatch_fwht_latency<MODE>(X, M, K, codes, scales, csum, Xr, s))
-    return launch_status();
+// Few tokens: more threads per token (8 or 16 values each) for latency; many
+// tokens: 32-128 values per thread for throughput.
+template <int MODE, bool IN_F32 = false, bool LN = false>
+int dispatch_fwht(const FwhtArgs& a, int K, cudaStream_t s) {
+  if (a.M <= kLatencyTokens) {
+    switch (ilog2(K)) {
+      case 10: launch_fwht<10, 3, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 11: launch_fwht<11, 3, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 12: launch_fwht<12, 3, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 13: launch_fwht<13, 3, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 14: launch_fwht<14, 4, MODE, IN_F32, LN>(a, s); return launch_status();
+      default: break;
+    }
+  }
   switch (ilog2(K)) {
-    case 8: launch_fwht<8, 4, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 9: launch_fwht<9, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 10: launch_fwht<10, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 11: launch_fwht<11, 6, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 12: launch_fwht<12, 6, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 13: launch_fwht<13, 7, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 14: launch_fwht<14, 7, MODE>(X, M, codes, scales, csum, Xr, s); break;
-    case 15: launch_fwht<15, 5, MODE>(X, M, codes, scales, csum, Xr, s); break;
+    case 8: launch_fwht<8, 4, MODE, IN_F32, LN>(a, s); break;
+    case 9: launch_fwht<9, 5, MODE, IN_F32, LN>(a, s); break;
+    case 10: launch_fwht<10, 5, MODE, IN_F32, LN>(a, s); break;
+    case 11: launch_fwht<11, 6, MODE, IN_F32, LN>(a, s); break;
+    case 12: launch_fwht<12, 6, MODE, IN_F32, LN>(a, s); break;
+    case 13: launch_fwht<13, 7, MODE, IN_F32, LN>(a, s); break;
+    case 14: launch_fwht<14, 7, MODE, IN_F32, LN>(a, s); break;
+    case 15: launch_fwht<15, 5, MODE, IN_F32, LN>(a, s); break;
     default: return HBL_ERR_SHAPE;
   }
   return launch_status();
 }
 
-template <int MODE>
-int dispatch_rows(const uint16_t* X, int M, int K, int8_t* codes, float* scales, int32_t* csum,
-                  cudaStream_t s) {
+template <int MODE, bool LN>
+int dispatch_rows(const uint16_t* X, int M, int K, const float* gain, int8_t* codes, float* scales,
+                  int32_t* csum, cudaStream_t s) {
   auto blocks = [](int T) { return (T + 31) / 32 * 32; };
   ProfScope ps("quant_rows", s);
   if (K <= 8192)
-    launch_pdl(quant_rows_kernel<8, MODE>, dim3(M), dim3(blocks(K / 8)), 0, s, X, M, K, codes, scales, csum);
+    launch_pdl(quant_rows_kernel<8, MODE, LN>, dim3(M), dim3(blocks(K / 8)), 0, s, X, M, K, gain, codes, scales,
+               csum);
   else if (K <= 16384)
-    launch_pdl(quant_rows_kernel<16, MODE>, dim3(M), dim3(blocks(K / 16)), 0, s, X, M, K, codes, scales, csum);
+    launch_pdl(quant_rows_kernel<16, MODE, LN>, dim3(M), dim3(blocks(K / 16)), 0, s, X, M, K, gain, codes, scales,
+               csum);
   else if (K <= 32768)
-    launch_pdl(quant_rows_kernel<32, MODE>, dim3(M), dim3(blocks(K / 32)), 0, s, X, M, K, codes, scales, csum);
+    launch_pdl(quant_rows_kernel<32, MODE, LN>, dim3(M), dim3(blocks(K / 32)), 0, s, X, M, K, gain, codes, scales,
+               csum);
   else
-    launch_pdl(quant_rows_kernel<64, MODE>, dim3(M), dim3(blocks(K / 64)), 0, s, X, M, K, codes, scales, csum);
+    launch_pdl(quant_rows_kernel<64, MODE, LN>, dim3(M), dim3(blocks(K / 64)), 0, s, X, M, K, gain, codes, scales,
+               csum);
   return launch_status();
 }
 
+// Optional RMSNorm (ln), optional Hadamard, then the per-token quantiser.
 int run_quantize(const uint16_t* X, int M, int K, int act_bits, int use_hadamard, int8_t* codes,
-                 float* scales, int32_t* csum, cudaStream_t s) {
+                 float* scales, int32_t* csum, cudaStream_t s, bool ln = false, const float* gain = nullptr) {
+  const FwhtArgs a{X, M, gain, codes, scales, csum, nullptr};
   if (use_hadamard) {
-    return act_bits == 4 ? dispatch_fwht<kModeInt4>(X, M, K, codes, scales, csum, nullptr, s)
-                         : dispatch_fwht<kModeInt8>(X, M, K, codes, scales, csum, nullptr, s);
+    if (ln)
+      return act_bits == 4 ? dispatch_fwht<kModeInt4, false, true>(a, K, s)
+                           : dispatch_fwht<kModeInt8, false, true>(a, K, s);
+    return act_bits == 4 ? dispatch_fwht<kModeInt4>(a, K, s) : dispatch_fwht<kModeInt8>(a, K, s);
   }
-  return act_bits == 4 ? dispatch_rows<kModeInt4>(X, M, K, codes, scales, csum, s)
-                       : dispatch_rows<kModeInt8>(X, M, K, codes, scales, csum, s);
+  if (ln)
+    return act_bits == 4 ? dispatch_rows<kModeInt4, true>(X, M, K, gain, codes, scales, csum, s)
+                         : dispatch_rows<kModeInt8, true>(X, M, K, gain, codes, scales, csum, s);
+  return act_bits == 4 ? dispatch_rows<kModeInt4, false>(X, M, K, nullptr, codes, scales, csum, s)
+                       : dispatch_rows<kModeInt8, false>(X, M, K, nullptr, codes, scales, csum, s);
 }
 
 // D = sum c*u over K. Chooses the token tile and a split of K so that the grid
@@ -409,7 +417,7 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 
 int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
                  int act_bits, int use_hadamard, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t s,
-                 DeviceState* d) {
+                 DeviceState* d, bool ln = false, const float* gain = nullptr) {
   const WsLayout L = ws_layout(M, K, N);
   if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return HBL_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
@@ -417,7 +425,7 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   float* scales = reinterpret_cast<float*>(base + L.scales);
   int32_t* csum = reinterpret_cast<int32_t*>(base + L.csum);
   int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
-  int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s);
+  int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
   if (st) return st;
   if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
   if (g_gemm_path != 1 && decode_path_fits(M, K))
@@ -555,7 +563,8 @@ int hbl_hadamard_f32(const hbl_bf16* X, int M, int K, float* Xr, hbl_stream stre
   if (misaligned16(X) || misaligned16(Xr)) return HBL_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   if ((st = ensure_device(&d))) return st;
-  return dispatch_fwht<kModeF32>(X, M, K, nullptr, nullptr, nullptr, Xr, reinterpret_cast<cudaStream_t>(stream));
+  return dispatch_fwht<kModeF32>(FwhtArgs{X, M, nullptr, nullptr, nullptr, nullptr, Xr}, K,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard, int8_t* codes, float* scales,
@@ -602,6 +611,80 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
     return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
   if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
   sub_rowsum_kernel<<<(unsigned)(((long long)M * N + 255) / 256), 256, 0, s>>>(acc, csum, M, N);
+  return launch_status();
+}
+
+int hbl_forward_ln_ws(const hbl_bf16* X, int M, int K, int N, const float* gain, const uint8_t* Wpk,
+                      const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y, void* ws, size_t ws_bytes,
+                      hbl_stream stream) {
+  int st = check_forward_args(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y);
+  if (st || M == 0) return st;
+  if (misaligned16(gain)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  return forward_impl(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, Y, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), d, true, gain);
+}
+
+int hbl_quantize_ln(const hbl_bf16* X, int M, int K, const float* gain, int act_bits, int use_hadamard,
+                    int8_t* codes, float* scales, int32_t* csum, hbl_stream stream) {
+  if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+  if (use_hadamard != 0 && use_hadamard != 1) return HBL_ERR_INVALID_ARG;
+  int st = check_act_shape(M, K, use_hadamard);
+  if (st || M == 0) return st;
+  if (!X || !codes || !scales) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(X) || misaligned16(codes) || misaligned16(gain)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  return run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, reinterpret_cast<cudaStream_t>(stream),
+                      true, gain);
+}
+
+int hbl_hadamard_backward_f32(const float* dXr, int M, int K, float* dX, hbl_stream stream) {
+  int st = check_act_shape(M, K, 1);
+  if (st || M == 0) return st;
+  if (!dXr || !dX) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(dXr) || misaligned16(dX)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  return dispatch_fwht<kModeF32, true, false>(FwhtArgs{dXr, M, nullptr, nullptr, nullptr, nullptr, dX}, K,
+                                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+int hbl_pack_weights_rotated(const float* W, int N, int K, uint8_t* Wpk, float* wscale, float* Wrot,
+                             hbl_stream stream) {
+  int st = check_weight_shape(N, K);
+  if (st) return st;
+  if ((st = check_act_shape(N, K, 1))) return st;
+  if (!W || !Wpk || !wscale || !Wrot) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(W) || misaligned16(Wpk) || misaligned16(Wrot)) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  if ((st = ensure_device(&d))) return st;
+  // every weight row w becomes H w (W H^T), in fp32, then the usual ternarise + pack
+  st = dispatch_fwht<kModeF32, true, false>(FwhtArgs{W, N, nullptr, nullptr, nullptr, nullptr, Wrot}, K,
+                                            reinterpret_cast<cudaStream_t>(stream));
+  if (st) return st;
+  return hbl_pack_weights(Wrot, N, K, Wpk, wscale, stream);
+}
+
+int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_token, uint8_t* codes,
+                     float* gamma, hbl_stream stream) {
+  if (T < 0 || H < 1 || (d != 64 && d != 128 && d != 256)) return HBL_ERR_SHAPE;
+  if ((long long)T * H >= (1ll << 31)) return HBL_ERR_SHAPE;
+  if (bits < 2 || bits > 8 || bos_token >= T) return HBL_ERR_INVALID_ARG;
+  if (T == 0) return HBL_OK;
+  if (!X || !codes || !gamma) return HBL_ERR_INVALID_ARG;
+  if (misaligned16(X) || misaligned16(codes)) return HBL_ERR_INVALID_ARG;
+  DeviceState* dev = nullptr;
+  int st = ensure_device(&dev);
+  if (st) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = T * H;
+  const dim3 grid((rows + 7) / 8);
+  ProfScope ps("qkv_quant", s);
+  if (d == 64) qkv_quant_kernel<2><<<grid, 256, 0, s>>>(X, rows, H, bits, bos_token, codes, gamma);
+  else if (d == 128) qkv_quant_kernel<4><<<grid, 256, 0, s>>>(X, rows, H, bits, bos_token, codes, gamma);
+  else qkv_quant_kernel<8><<<grid, 256, 0, s>>>(X, rows, H, bits, bos_token, codes, gamma);
   return launch_status();
 }
 

@@ -31,6 +31,11 @@ SIGNATURES = [
     ("hbl_hadamard_f32", _I, [_P, _I, _I, _P, _P]),
     ("hbl_quantize", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _P]),
     ("hbl_gemm_codes", _I, [_P, _I, _I, _I, _P, _P, _P]),
+    ("hbl_forward_ln_ws", _I, [_P, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _Z, _P]),
+    ("hbl_quantize_ln", _I, [_P, _I, _I, _P, _I, _I, _P, _P, _P, _P]),
+    ("hbl_pack_weights_rotated", _I, [_P, _I, _I, _P, _P, _P, _P]),
+    ("hbl_hadamard_backward_f32", _I, [_P, _I, _I, _P, _P]),
+    ("hbl_quantize_qkv", _I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     ("hbl_get_device_error", _I, [_P]),
     ("hbl_set_gemm_path", _I, [_I]),
     ("hbl_profile_enable", _I, [_I]),
@@ -136,6 +141,32 @@ def hbl_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum=None, stre
 def hbl_gemm_codes(codes, M, K, N, Wpk, acc, stream=None):
     return _check(lib().hbl_gemm_codes(_ptr(codes), M, K, N, _ptr(Wpk), _ptr(acc), _stream(stream)),
                   "hbl_gemm_codes")
+
+
+def hbl_forward_ln_ws(X, M, K, N, gain, Wpk, wscale, act_bits, use_hadamard, Y, ws, ws_bytes, stream=None):
+    return _check(lib().hbl_forward_ln_ws(_ptr(X), M, K, N, _ptr(gain), _ptr(Wpk), _ptr(wscale), act_bits,
+                                          use_hadamard, _ptr(Y), _ptr(ws), ws_bytes, _stream(stream)),
+                  "hbl_forward_ln_ws")
+
+
+def hbl_quantize_ln(X, M, K, gain, act_bits, use_hadamard, codes, scales, csum=None, stream=None):
+    return _check(lib().hbl_quantize_ln(_ptr(X), M, K, _ptr(gain), act_bits, use_hadamard, _ptr(codes),
+                                        _ptr(scales), _ptr(csum), _stream(stream)), "hbl_quantize_ln")
+
+
+def hbl_pack_weights_rotated(W, N, K, Wpk, wscale, Wrot, stream=None):
+    return _check(lib().hbl_pack_weights_rotated(_ptr(W), N, K, _ptr(Wpk), _ptr(wscale), _ptr(Wrot),
+                                                 _stream(stream)), "hbl_pack_weights_rotated")
+
+
+def hbl_hadamard_backward_f32(dXr, M, K, dX, stream=None):
+    return _check(lib().hbl_hadamard_backward_f32(_ptr(dXr), M, K, _ptr(dX), _stream(stream)),
+                  "hbl_hadamard_backward_f32")
+
+
+def hbl_quantize_qkv(X, T, H, d, bits, bos_token, codes, gamma, stream=None):
+    return _check(lib().hbl_quantize_qkv(_ptr(X), T, H, d, bits, bos_token, _ptr(codes), _ptr(gamma),
+                                         _stream(stream)), "hbl_quantize_qkv")
 
 
 def hbl_get_device_error(stream=None):

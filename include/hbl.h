@@ -186,6 +186,63 @@ int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard
 int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
                    int32_t* acc, hbl_stream stream);
 
+/* ------------------------------------------------------------------------
+ * Beyond the LN-free forward: the LN of Eq. 9, the rotated-weight variant,
+ * the Hadamard backward (Eq. 10) and the post-RoPE QKV quantiser.
+ * ------------------------------------------------------------------------ */
+
+/*
+ * hbl_forward_ln_ws -- the full H-BitLinear of Eq. 9 (section 3.4, "H-BitLinear:
+ * The Composite Layer"): X_r = Hadamard(LN(X)) with LN the RMSNorm
+ *   LN(x) = x * gain / sqrt(mean(x^2) + 1e-5)
+ * (the epsilon is a reading: the pages give none). gain: device fp32 K, or
+ * NULL for no gain. Everything else as hbl_forward_ws (same workspace size).
+ * The normalisation is fused into the Hadamard/quantise kernel: the gain is
+ * applied on load and the per-token factor is folded into the transform's
+ * final scaling.
+ */
+int hbl_forward_ln_ws(const hbl_bf16* X, int M, int K, int N, const float* gain, const uint8_t* Wpk,
+                      const float* wscale, int act_bits, int use_hadamard, hbl_bf16* Y, void* ws,
+                      size_t ws_bytes, hbl_stream stream);
+
+/* hbl_quantize_ln -- hbl_quantize with the RMSNorm above applied first. */
+int hbl_quantize_ln(const hbl_bf16* X, int M, int K, const float* gain, int act_bits,
+                    int use_hadamard, int8_t* codes, float* scales, int32_t* csum, hbl_stream stream);
+
+/*
+ * hbl_pack_weights_rotated -- the weight-and-activation rotation variant of the
+ * ablation in section 3.4 (Table 5): packs Q_w(W H^T), i.e. every weight row w
+ * is replaced by H w (fp32) before the ternary quantiser of Eq. 1-2. Used with
+ * use_hadamard = 1 in the forward, the product is Q_w(W H^T) . Q(H x).
+ *   Wrot : device fp32 N x K caller scratch; receives W H^T.
+ * K must be a power of two, 256 <= K <= 32768; otherwise as hbl_pack_weights.
+ */
+int hbl_pack_weights_rotated(const float* W, int N, int K, uint8_t* Wpk, float* wscale,
+                             float* Wrot, hbl_stream stream);
+
+/*
+ * hbl_hadamard_backward_f32 -- Eq. 10 (section 3.4, "Gradient Handling Through
+ * the Hadamard Transformation"): dL/dX = H^T dL/dX_r per token, which for the
+ * symmetric Sylvester H is the same fast transform. fp32 in, fp32 out, M x K.
+ * K must be a power of two, 256 <= K <= 32768.
+ */
+int hbl_hadamard_backward_f32(const float* dXr, int M, int K, float* dX, hbl_stream stream);
+
+/*
+ * hbl_quantize_qkv -- post-RoPE QKV quantiser (section 3.4, "QKV Attention
+ * Quantization"): each head vector of d values is quantised to unsigned
+ * b-bit integers from its absmax gamma. Reading of "unsigned absmax":
+ *   u = RoundClip((2^b - 1)/2 * (x / (gamma + 1e-5) + 1), 0, 2^b - 1),
+ *   dequantised value (2u / (2^b - 1) - 1) * gamma.
+ * The heads of token `bos_token` (the BOS token; -1 for none) use 8 bits.
+ *   X     : device bf16, T x H x d (token, head, channel).
+ *   codes : device uint8, T x H x d, one code per byte.
+ *   gamma : device fp32, T x H.
+ * d in {64, 128, 256}; 2 <= bits <= 8.
+ */
+int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_token,
+                     uint8_t* codes, float* gamma, hbl_stream stream);
+
 /*
  * hbl_get_device_error -- synchronises `stream`, then reads and clears the
  * device error word that bounded waits inside the kernels set when they give
