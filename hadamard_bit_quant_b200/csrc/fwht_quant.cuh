@@ -12,8 +12,8 @@
 // index bits, processed top-down. In a pass that owns bits [lo, lo+G), thread
 // t holds the E values whose indices differ only in those bits, and the
 // butterflies run in registers. Between passes the values are exchanged
-// through shared memory (an XOR swizzle keeps both access patterns free of
-// bank conflicts). The first pass owns the top bits, so its loads are
+// through shared memory (one pad word per 2^G values keeps every access
+// pattern free of bank conflicts). The first pass owns the top bits, so its loads are
 // coalesced across threads; the last pass owns bits [0, G), so each thread
 // ends with E consecutive values and stores E consecutive codes.
 #pragma once
@@ -32,7 +32,8 @@ struct FwhtCfg {
   static constexpr int THREADS = T * TPC;
   static constexpr int P = (LOG_K + G - 1) / G;         // passes
   static constexpr int WARPS_PER_TOKEN = T >= 32 ? T / 32 : 1;
-  static constexpr size_t SMEM = (size_t)TPC * K * sizeof(float);
+  static constexpr int KPAD = K + K / E;                 // one pad word per E values
+  static constexpr size_t SMEM = (size_t)TPC * KPAD * sizeof(float);
 };
 
 template <int G>
@@ -42,8 +43,13 @@ HBL_DEVINL int pass_index(int t, int j, int lo) {
   return low | (j << lo) | (high << (lo + G));
 }
 
+// Shared-memory position of index idx: one pad word after every 2^G values.
+// For every exchange pattern used here (32 consecutive threads, one register
+// index) the padded positions fall in 32 distinct banks, and because the
+// thread part and the register part of idx occupy disjoint bits, the
+// position splits into (thread part) + (compile-time offset per register).
 template <int G>
-HBL_DEVINL int swz(int idx) { return idx ^ ((idx >> G) & 31); }
+HBL_DEVINL int pad(int idx) { return idx + (idx >> G); }
 
 // Sum / max over the T threads of one token. Threads of a token are T
 // consecutive lanes (T < 32) or T/32 whole warps (T >= 32). `red` holds one
@@ -91,12 +97,22 @@ HBL_DEVINL int token_reduce_i(int x, int* red, int token_sub) {
 
 // Quantise E consecutive values v[] of a token whose T threads hold the whole
 // row (K values), write codes / scale / code sum, or the fp32 values (kModeF32).
+// v holds the values before the scale `nrm` (> 0) of the transform is applied:
+// X_r = nrm * v. The scale is applied to the statistic and folded into the
+// quantiser's multiplier, so each value is multiplied once.
 template <int E, int T, int WPT, int MODE>
 HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool active, size_t m,
                            float* red_f, int* red_i, int8_t* __restrict__ codes,
                            float* __restrict__ scales, int32_t* __restrict__ csum,
-                           float* __restrict__ Xr) {
+                           float* __restrict__ Xr, float nrm = 1.f) {
   if constexpr (MODE == kModeF32) {
+    const float2 n2 = make_float2(nrm, nrm);
+#pragma unroll
+    for (int j = 0; j < E; j += 2) {
+      const float2 r = __fmul2_rn(make_float2(v[j], v[j + 1]), n2);
+      v[j] = r.x;
+      v[j + 1] = r.y;
+    }
     if (active) {
       float4* dst = reinterpret_cast<float4*>(Xr + m * (size_t)K + (size_t)E * t);
 #pragma unroll
@@ -112,7 +128,7 @@ HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool acti
 #pragma unroll
       for (int j = 0; j < E; ++j) part = fmaxf(part, fabsf(v[j]));
     }
-    const float r = token_reduce_f<T, WPT, MODE == kModeInt8>(part, red_f, token_sub);
+    const float r = __fmul_rn(token_reduce_f<T, WPT, MODE == kModeInt8>(part, red_f, token_sub), nrm);
     float mult, scale;
     int lo, hi;
     if constexpr (MODE == kModeInt4) {
@@ -125,6 +141,7 @@ HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool acti
       scale = __fdiv_rn(r, 127.f);
       lo = -128; hi = 127;
     }
+    mult = __fmul_rn(mult, nrm);
     int cs = 0;
     uint32_t packed[E / 4];
 #pragma unroll
@@ -210,7 +227,7 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
   const int t = threadIdx.x % T;
   const size_t m = (size_t)blockIdx.x * C::TPC + token_sub;
   const bool active = m < (size_t)M;
-  float* sm = smem + (size_t)token_sub * K;
+  float* sm = smem + (size_t)token_sub * C::KPAD;
 
   // Programmatic dependent launch: let the consumer grid launch now (it only
   // prefetches weights until this grid completes), and wait for the producer
@@ -246,10 +263,10 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
       const int hi_prev = LOG_K - (p - 1) * G;
       const int lo_prev = hi_prev - G > 0 ? hi_prev - G : 0;
 #pragma unroll
-      for (int j = 0; j < E; ++j) sm[swz<G>(pass_index<G>(t, j, lo_prev))] = v[j];
+      for (int j = 0; j < E; ++j) sm[pad<G>(pass_index<G>(t, j, lo_prev))] = v[j];
       __syncthreads();
 #pragma unroll
-      for (int j = 0; j < E; ++j) v[j] = sm[swz<G>(pass_index<G>(t, j, lo))];
+      for (int j = 0; j < E; ++j) v[j] = sm[pad<G>(pass_index<G>(t, j, lo))];
       if (p + 1 < P) __syncthreads();
     }
     butterflies<E>(v, nb);
@@ -263,16 +280,9 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
       const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)K), kRmsEps)));
       nrm = __fmul_rn(nrm, r);
     }
-    const float2 n2 = make_float2(nrm, nrm);
-#pragma unroll
-    for (int j = 0; j < E; j += 2) {
-      const float2 r = __fmul2_rn(make_float2(v[j], v[j + 1]), n2);
-      v[j] = r.x;
-      v[j + 1] = r.y;
-    }
+    quant_tail<E, T, C::WARPS_PER_TOKEN, MODE>(v, K, t, token_sub, active, m, red_f, red_i, codes,
+                                               scales, csum, Xr, nrm);
   }
-  quant_tail<E, T, C::WARPS_PER_TOKEN, MODE>(v, K, t, token_sub, active, m, red_f, red_i, codes,
-                                             scales, csum, Xr);
 }
 
 // Plain per-token quantiser (no Hadamard), K % 256 == 0, one token per CTA,

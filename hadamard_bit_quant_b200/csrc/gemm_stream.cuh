@@ -1,0 +1,290 @@
+// Weight-streaming ternary x int8 GEMM for the decode regime (1..16 tokens),
+// with the dequant epilogue fused.
+//
+// BitNet v2 architecture walkthrough, section 3.4 "H-BitLinear: The Composite
+// Layer", Eq. 9: acc[m, n] = sum_k c[m, k] * t[n, k]; Y = acc * s[m] * alpha.
+//
+// With few tokens the forward moves N*K/4 bytes of packed weights and little
+// else, so the kernel is built to keep HBM busy:
+//   * one CTA per SM (persistent); CTA c owns the 16-row groups c, c+G, ...
+//     over the whole of K, so no partial sums ever leave the CTA;
+//   * K is walked in chunks of 2048; a chunk's codes (M x 2048 int8) sit in
+//     one of two shared-memory buffers, loaded once per chunk by TMA;
+//   * the weights of each (chunk, group) unit -- 16 rows x 512 bytes -- stream
+//     through a 16-stage TMA ring (128 KB in flight per SM). The ring is
+//     filled before the kernel waits for the quantiser grid (programmatic
+//     dependent launch), so a layer's weights arrive while the previous
+//     kernel still runs;
+//   * 8 consumer warps take one 256-k block of each unit each: weights as the
+//     m16n8k32 A operand (u = t + 1 unpacked in registers), codes as B, both
+//     from 128B-swizzled shared memory (conflict-free), accumulating in
+//     registers across chunks; a dedicated producer warp issues the copies;
+//   * at the end the 8 warps' partial sums are added in shared memory, the
+//     code sums subtracted, scaled and stored as bf16 (or int32).
+// Every mbarrier wait is bounded; a CTA that gives up sets the device error
+// word, lets its outstanding copies land (bounded) and exits.
+#pragma once
+#include <cuda.h>
+#include "hbl_common.cuh"
+#include "gemm_mma.cuh"
+
+namespace hbl {
+namespace strm {
+
+constexpr int kGroupRows = 16;
+constexpr int kChunk = 2048;                       // k per chunk
+constexpr int kBlocksPerChunk = kChunk / kKBlock;  // 8 = one per consumer warp
+constexpr int kConsumers = 8;
+constexpr int kThreads = 32 * (kConsumers + 1);
+#ifndef HBL_STREAM_STAGES
+#define HBL_STREAM_STAGES 16
+#endif
+constexpr int kStages = HBL_STREAM_STAGES;
+constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB: 4 boxes of [16][128 B]
+constexpr int kMaxGroups = 8;                      // per CTA
+constexpr long long kSpinLimit = 4000000000ll;
+
+HBL_DEVINL uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+HBL_DEVINL void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(su32(b)), "r"(count) : "memory");
+}
+HBL_DEVINL void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+HBL_DEVINL void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(su32(b)) : "memory");
+}
+HBL_DEVINL bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+HBL_DEVINL bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(b, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kSpinLimit) {
+      *abort = 1;
+      set_device_error(HBL_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+HBL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
+          su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+template <int MT>
+struct Layout {
+  static constexpr int kCodeBox = MT * 128;                 // one [MT][128 B] box
+  static constexpr int kCodeBuf = (kChunk / 128) * kCodeBox;
+  static constexpr size_t kRing = (size_t)kStages * kUnitBytes;
+  static constexpr size_t kBytes = 1024 + kRing + 2 * (size_t)kCodeBuf + 256;
+};
+
+template <int TN, bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_c,
+                   const int32_t* __restrict__ csum, const float* __restrict__ scales,
+                   const float* __restrict__ alpha, int M, int K, int N, uint16_t* __restrict__ Y,
+                   int32_t* __restrict__ acc_out) {
+  constexpr int MT = 8 * TN;
+  using Lay = Layout<MT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = base;
+  uint8_t* cbuf = ring + Lay::kRing;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cbuf + 2 * Lay::kCodeBuf);
+  uint64_t* wfull = bars;                 // [kStages]
+  uint64_t* wempty = bars + kStages;      // [kStages]
+  uint64_t* cfull = bars + 2 * kStages;   // [2]
+  uint64_t* cempty = cfull + 2;           // [2]
+  volatile int* abort = reinterpret_cast<volatile int*>(cempty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int groups = N / kGroupRows;
+  const int G = gridDim.x;
+  const int ng = (groups - (int)blockIdx.x + G - 1) / G;    // groups owned by this CTA
+  const int nchunks = K / kChunk;
+  const int units = nchunks * ng;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], kConsumers);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&cfull[b], 1);
+      mbar_init(&cempty[b], kConsumers);
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumers) {
+    // ----- producer -----
+    if (lane == 0) {
+      auto issue_w = [&](int u) {
+        const int s = u % kStages;
+        const int c = u / ng, gl = u % ng;
+        const int row0 = ((int)blockIdx.x + gl * G) * kGroupRows;
+        mbar_expect_tx(&wfull[s], kUnitBytes);
+        uint8_t* dst = ring + (size_t)s * kUnitBytes;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(dst + b * (kGroupRows * 128), &map_w, &wfull[s], c * (kChunk / 4) + b * 128, row0);
+      };
+      auto issue_c = [&](int c) {
+        uint8_t* dst = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
+        mbar_expect_tx(&cfull[c & 1], (uint32_t)Lay::kCodeBuf);
+        for (int b = 0; b < kChunk / 128; ++b) tma_load_2d(dst + b * Lay::kCodeBox, &map_c, &cfull[c & 1], c * kChunk + b * 128, 0);
+      };
+      int u = 0;
+      for (; u < units && u < kStages; ++u) issue_w(u);             // weights do not depend on the previous grid
+      asm volatile("griddepcontrol.wait;\n" ::: "memory");          // codes do
+      int issued_c = 0;
+      if (nchunks > 0) { issue_c(0); issued_c = 1; }
+      bool ok = true;
+      // Codes run one chunk ahead of the weight units: chunk c+1's codes are
+      // requested as soon as the consumers have started chunk c-1 (its buffer
+      // is then free), before chunk c's remaining weight units.
+      for (int c = 0; c < nchunks && ok; ++c) {
+        if (c + 1 < nchunks) {
+          if (c + 1 >= 2 && !mbar_wait(&cempty[(c + 1) & 1], (uint32_t)(((c + 1) >> 1) - 1) & 1u, abort)) {
+            ok = false;
+            break;
+          }
+          issue_c(c + 1);
+          issued_c = c + 2;
+        }
+        for (; u < units && u < (c + 1) * ng; ++u) {
+          const int s = u % kStages;
+          if (!mbar_wait(&wempty[s], (uint32_t)((u / kStages) - 1) & 1u, abort)) { ok = false; break; }
+          issue_w(u);
+        }
+      }
+      // bounded drain of the copies issued last
+      const int last = u;
+      for (int q = (last > kStages ? last - kStages : 0); q < last; ++q) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&wfull[q % kStages], (uint32_t)(q / kStages) & 1u) && clock64() - t0 < kSpinLimit) {
+        }
+      }
+      for (int c = (issued_c > 2 ? issued_c - 2 : 0); c < issued_c; ++c) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&cfull[c & 1], (uint32_t)(c >> 1) & 1u) && clock64() - t0 < kSpinLimit) {
+        }
+      }
+    }
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  } else {
+    // ----- consumers: warp w takes 256-k block w of every unit -----
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    const int g = lane >> 2, tig = lane & 3;
+    int acc[kMaxGroups][TN][4];
+#pragma unroll
+    for (int a = 0; a < kMaxGroups; ++a)
+#pragma unroll
+      for (int i = 0; i < TN; ++i)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
+    bool ok = true;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&cfull[c & 1], (uint32_t)(c >> 1) & 1u, abort))) { ok = false; break; }
+      const uint8_t* cb = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
+      // B fragments of this warp's block for this chunk (reused by every group)
+      uint2 bf[TN][8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int box = 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
+#pragma unroll
+        for (int i = 0; i < TN; ++i) {
+          const int m = 8 * i + g;
+          bf[i][q] = *reinterpret_cast<const uint2*>(cb + box * Lay::kCodeBox + m * 128 + ((cch ^ (m & 7)) << 4) +
+                                                     ((tig & 1) << 3));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
+#pragma unroll
+      for (int gl = 0; gl < kMaxGroups; ++gl) {
+        if (gl < ng) {
+          const int u = c * ng + gl;
+          const int s = u % kStages;
+          if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) { ok = false; break; }
+          const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
+          const int ch = ((warp & 1) << 2) + tig;
+          const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
+          const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&wempty[s]);
+          const uint32_t A4[4] = {pa.x, pa.y, pa.z, pa.w};
+          const uint32_t B4[4] = {pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int w = q >> 1, jj = 2 * (q & 1);
+            const uint32_t a[4] = {unpack_u8x4(A4[w], jj), unpack_u8x4(B4[w], jj), unpack_u8x4(A4[w], jj + 1),
+                                   unpack_u8x4(B4[w], jj + 1)};
+#pragma unroll
+            for (int i = 0; i < TN; ++i) mma_u8s8_16832(acc[gl][i], a, bf[i][q].x, bf[i][q].y);
+          }
+        }
+      }
+    }
+    // partial sums of the 8 warps -> shared memory (aliases the ring, so only
+    // after every warp is done with it): red[warp][group][row][token]
+    asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers * 32) : "memory");
+    if (ok && *abort == 0) {
+      int* red = reinterpret_cast<int*>(ring);
+#pragma unroll
+      for (int gl = 0; gl < kMaxGroups; ++gl) {
+        if (gl < ng) {
+#pragma unroll
+          for (int i = 0; i < TN; ++i)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int row = g + ((r >> 1) << 3);
+              const int tok = 8 * i + 2 * tig + (r & 1);
+              red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
+            }
+        }
+      }
+    }
+  }
+  // every copy was consumed (or the CTA gave up); the ring may be reused
+  const bool all_ok = __syncthreads_and(*abort == 0) != 0;
+  if (all_ok && warp < kConsumers) {
+    const int* red = reinterpret_cast<const int*>(ring);
+    const float a = OUT_BF16 ? __ldg(alpha) : 0.f;
+    const int per_group = kGroupRows * MT;
+    for (int e = threadIdx.x; e < ng * per_group; e += kConsumers * 32) {
+      const int gl = e / per_group, rem = e % per_group;
+      const int tok = rem / kGroupRows, row = rem % kGroupRows;
+      const int n = ((int)blockIdx.x + gl * G) * kGroupRows + row;
+      if (tok < M) {
+        int s = 0;
+#pragma unroll
+        for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * kGroupRows + row) * MT + tok];
+        s -= __ldg(csum + tok);
+        if constexpr (OUT_BF16) {
+          const float y = __fmul_rn(__fmul_rn((float)s, __ldg(scales + tok)), a);
+          Y[(size_t)tok * N + n] = float_to_bf16_bits(y);
+        } else {
+          acc_out[(size_t)tok * N + n] = s;
+        }
+      }
+    }
+  }
+}
+
+}  // namespace strm
+}  // namespace hbl

@@ -14,7 +14,10 @@
 #include "fwht_quant.cuh"
 #include "gemm_mma.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "gemm_decode.cuh"
+#include "gemm_decode2.cuh"
+#include "gemm_stream.cuh"
 #include "qkv_quant.cuh"
 
 namespace hbl {
@@ -173,6 +176,11 @@ int check_act_shape(int M, int K, int use_hadamard) {
   return HBL_OK;
 }
 
+#ifndef HBL_USE_PDL
+#define HBL_USE_PDL 1
+#endif
+constexpr bool kUsePdl = HBL_USE_PDL != 0;
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel in the stream drains; it must execute griddepcontrol.wait
 // before touching anything that kernel writes.
@@ -188,23 +196,31 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kUsePdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
 // Raise a kernel's dynamic shared memory limit once per device (needed above 48 KB).
+// The limit recorded per (device, kernel) only ever grows.
 template <typename F>
 void ensure_smem_attr(F* func, size_t bytes) {
   if (bytes <= 48 * 1024) return;
+  struct Entry { int dev; const void* fn; size_t bytes; };
   static std::mutex mu;
-  static std::vector<std::pair<int, const void*>> done;
+  static std::vector<Entry> done;
   int dev = 0;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(mu);
-  for (auto& e : done)
-    if (e.first == dev && e.second == (const void*)func) return;
+  for (auto& e : done) {
+    if (e.dev == dev && e.fn == (const void*)func) {
+      if (e.bytes >= bytes) return;
+      cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+      e.bytes = bytes;
+      return;
+    }
+  }
   cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  done.emplace_back(dev, (const void*)func);
+  done.push_back(Entry{dev, (const void*)func, bytes});
 }
 
 // Arguments of one Hadamard(+quantise) launch.
@@ -229,6 +245,9 @@ void launch_fwht(const FwhtArgs& a, cudaStream_t s) {
 }
 
 constexpr int kLatencyTokens = 64;
+#ifndef HBL_FWHT_LAT_G12
+#define HBL_FWHT_LAT_G12 3
+#endif
 
 // Few tokens: more threads per token (8 or 16 values each) for latency; many
 // tokens: 32-128 values per thread for throughput.
@@ -238,7 +257,7 @@ int dispatch_fwht(const FwhtArgs& a, int K, cudaStream_t s) {
     switch (ilog2(K)) {
       case 10: launch_fwht<10, 3, MODE, IN_F32, LN>(a, s); return launch_status();
       case 11: launch_fwht<11, 3, MODE, IN_F32, LN>(a, s); return launch_status();
-      case 12: launch_fwht<12, 3, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 12: launch_fwht<12, HBL_FWHT_LAT_G12, MODE, IN_F32, LN>(a, s); return launch_status();
       case 13: launch_fwht<13, 3, MODE, IN_F32, LN>(a, s); return launch_status();
       case 14: launch_fwht<14, 4, MODE, IN_F32, LN>(a, s); return launch_status();
       default: break;
@@ -363,12 +382,38 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
-int g_gemm_path = 0;  // 0 auto, 1 warp-level mma.sync, 2 tcgen05
+// 0 auto, 1 warp-level mma.sync, 2 tcgen05 persistent (128 x 128 tiles), 3 decode without
+// clusters or streaming, 4 tcgen05 one 128 x 256 tile per CTA (the default for M >= 128),
+// 5 weight-streaming decode (the default for M <= 16 where it fits)
+int g_gemm_path = 0;
 
 bool use_tc_path(int M) {
   if (g_gemm_path == 1) return false;
-  if (g_gemm_path == 2) return true;
+  if (g_gemm_path == 2 || g_gemm_path == 4) return true;
   return M >= 128;
+}
+
+// Persistent tcgen05 kernel (one CTA per SM, 128 x 128 tiles, double-buffered accumulator).
+int run_gemm_tc2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
+                 const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count,
+                 cudaStream_t s) {
+  CUtensorMap mc, mw;
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc2::kToks, true)) return HBL_ERR_CUDA;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc2::kRows, false))
+    return HBL_ERR_CUDA;
+  const int tiles = ((N + tc2::kRows - 1) / tc2::kRows) * ((M + tc2::kToks - 1) / tc2::kToks);
+  const dim3 grid(tiles < sm_count ? tiles : sm_count);
+  ProfScope ps("gemm_tc", s);
+  if (Y) {
+    ensure_smem_attr(tc2::gemm_tc2_kernel<true>, tc2::kSmemBytes);
+    tc2::gemm_tc2_kernel<true><<<grid, tc2::kThreads, tc2::kSmemBytes, s>>>(mc, mw, M, K, N, csum, scales, alpha,
+                                                                            Y, nullptr);
+  } else {
+    ensure_smem_attr(tc2::gemm_tc2_kernel<false>, tc2::kSmemBytes);
+    tc2::gemm_tc2_kernel<false><<<grid, tc2::kThreads, tc2::kSmemBytes, s>>>(mc, mw, M, K, N, csum, nullptr,
+                                                                             nullptr, nullptr, acc);
+  }
+  return launch_status();
 }
 
 // bf16 output (Y != nullptr) or int32 output (acc != nullptr); D - csum either way.
@@ -393,8 +438,128 @@ bool decode_path_fits(int M, int K) {
   return M <= kLatencyTokens && dec::smem_bytes(K, 8) <= 200 * 1024;
 }
 
+#ifndef HBL_DECODE_MAX_CLUSTER
+#define HBL_DECODE_MAX_CLUSTER 8
+#endif
+constexpr int kDecodeMaxCluster = HBL_DECODE_MAX_CLUSTER;
+
+// Cluster K-split decode kernel: cluster size C (K slice KC = K / C) and shared memory.
+bool decode2_config(int M, int K, int* C_out, int* KC_out, size_t* smem_out) {
+  // measured on B200: below 9 tokens the one-CTA-per-16-rows kernel is faster
+  if (M > kLatencyTokens || M <= 8 || K < 512) return false;
+  const int MT = 8 * (M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8)));
+  for (int C = kDecodeMaxCluster; C >= 1; C >>= 1) {
+    if (K % C) continue;
+    const int KC = K / C;
+    if (KC % 512) continue;
+    const size_t sm = dec2::smem_bytes(KC, MT);
+    if (sm <= 200 * 1024) {
+      *C_out = C;
+      *KC_out = KC;
+      *smem_out = sm;
+      return true;
+    }
+  }
+  return false;
+}
+
+int run_gemm_decode2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
+                     const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
+  int C = 0, KC = 0;
+  size_t smem = 0;
+  if (!decode2_config(M, K, &C, &KC, &smem)) return HBL_ERR_UNSUPPORTED;
+  const int TN = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
+  CUtensorMap mw, mc;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, dec2::kRows, true))
+    return HBL_ERR_CUDA;
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), true))
+    return HBL_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, (N + dec2::kRows - 1) / dec2::kRows);
+  cfg.blockDim = dim3(dec2::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kUsePdl ? 2 : 1;
+  ProfScope ps("gemm_decode", s);
+  cudaError_t e = cudaSuccess;
+#define HBL_DEC2(TN_)                                                                                         \
+  if (Y) {                                                                                                    \
+    ensure_smem_attr(dec2::gemm_decode_cluster_kernel<TN_, true>, smem);                                      \
+    e = cudaLaunchKernelEx(&cfg, dec2::gemm_decode_cluster_kernel<TN_, true>, mw, mc, csum, scales, alpha, M, K, \
+                           N, KC, Y, (int32_t*)nullptr);                                                      \
+  } else {                                                                                                    \
+    ensure_smem_attr(dec2::gemm_decode_cluster_kernel<TN_, false>, smem);                                     \
+    e = cudaLaunchKernelEx(&cfg, dec2::gemm_decode_cluster_kernel<TN_, false>, mw, mc, csum,                  \
+                           (const float*)nullptr, (const float*)nullptr, M, K, N, KC, (uint16_t*)nullptr, acc); \
+  }
+  switch (TN) {
+    case 1: HBL_DEC2(1); break;
+    case 2: HBL_DEC2(2); break;
+    case 4: HBL_DEC2(4); break;
+    default: HBL_DEC2(8); break;
+  }
+#undef HBL_DEC2
+  return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
+}
+
+// Weight-streaming decode kernel: M <= 16, K % 2048 == 0, at most 8 row groups per CTA.
+bool stream_fits(int M, int K, int N, int sm_count) {
+  if (M < 1 || M > 16 || K % strm::kChunk != 0) return false;
+  const int groups = N / strm::kGroupRows;
+  const int G = groups < sm_count ? groups : sm_count;
+  return G > 0 && groups <= strm::kMaxGroups * G;
+}
+
+int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
+                    const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count,
+                    cudaStream_t s) {
+  const int TN = M <= 8 ? 1 : 2;
+  CUtensorMap mw, mc;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, strm::kGroupRows, true))
+    return HBL_ERR_CUDA;
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), true))
+    return HBL_ERR_CUDA;
+  const int groups = N / strm::kGroupRows;
+  const dim3 grid(groups < sm_count ? groups : sm_count);
+  ProfScope ps("gemm_decode", s);
+  cudaError_t e;
+#define HBL_STRM(TN_)                                                                                          \
+  {                                                                                                            \
+    const size_t sm = strm::Layout<8 * TN_>::kBytes;                                                           \
+    if (Y) {                                                                                                   \
+      ensure_smem_attr(strm::gemm_stream_kernel<TN_, true>, sm);                                               \
+      e = launch_pdl(strm::gemm_stream_kernel<TN_, true>, grid, dim3(strm::kThreads), sm, s, mw, mc, csum,      \
+                     scales, alpha, M, K, N, Y, (int32_t*)nullptr);                                            \
+    } else {                                                                                                   \
+      ensure_smem_attr(strm::gemm_stream_kernel<TN_, false>, sm);                                              \
+      e = launch_pdl(strm::gemm_stream_kernel<TN_, false>, grid, dim3(strm::kThreads), sm, s, mw, mc, csum,     \
+                     (const float*)nullptr, (const float*)nullptr, M, K, N, (uint16_t*)nullptr, acc);          \
+    }                                                                                                          \
+  }
+  if (TN == 1) HBL_STRM(1) else HBL_STRM(2)
+#undef HBL_STRM
+  return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
+}
+
 int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
-                    const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
+                    const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s,
+                    int sm_count = 148) {
+  if ((g_gemm_path == 0 || g_gemm_path == 5) && stream_fits(M, K, N, sm_count))
+    return run_gemm_stream(codes, M, K, N, Wpk, csum, scales, alpha, Y, acc, sm_count, s);
+  {
+    int C, KC;
+    size_t sm;
+    if (g_gemm_path != 3 && decode2_config(M, K, &C, &KC, &sm))
+      return run_gemm_decode2(codes, M, K, N, Wpk, csum, scales, alpha, Y, acc, s);
+  }
   const int TN = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
   const dim3 grid((N + dec::kRows - 1) / dec::kRows);
   const size_t smem = dec::smem_bytes(K, TN);
@@ -427,9 +592,11 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
   if (st) return st;
-  if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
+  if (use_tc_path(M))
+    return g_gemm_path == 2 ? run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s)
+                            : run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
   if (g_gemm_path != 1 && decode_path_fits(M, K))
-    return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
+    return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count);
   st = run_gemm(codes, M, K, N, Wpk, D, d->sm_count, s);
   if (st) return st;
   const long long total8 = (long long)M * N / 8;
@@ -606,9 +773,11 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   }
   code_rowsum_kernel<<<M, 256, 0, s>>>(codes, K, csum);
   if ((st = launch_status())) return st;
-  if (use_tc_path(M)) return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
+  if (use_tc_path(M))
+    return g_gemm_path == 2 ? run_gemm_tc2(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s)
+                            : run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
   if (g_gemm_path != 1 && decode_path_fits(M, K))
-    return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
+    return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count);
   if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
   sub_rowsum_kernel<<<(unsigned)(((long long)M * N + 255) / 256), 256, 0, s>>>(acc, csum, M, N);
   return launch_status();
@@ -689,7 +858,7 @@ int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_t
 }
 
 int hbl_set_gemm_path(int path) {
-  if (path < 0 || path > 2) return HBL_ERR_INVALID_ARG;
+  if (path < 0 || path > 5) return HBL_ERR_INVALID_ARG;
   g_gemm_path = path;
   return HBL_OK;
 }

@@ -253,10 +253,17 @@ int hbl_get_device_error(hbl_stream stream);
 
 /*
  * hbl_set_gemm_path -- which integer-GEMM kernel the forward and
- * hbl_gemm_codes use: 0 = by size (default: tcgen05 tensor-core kernel for
- * M >= 128 tokens, warp-level mma.sync kernel below), 1 = always the
- * warp-level kernel, 2 = always the tcgen05 kernel. Both give identical
- * results; the knob exists to check and time each one. Process-wide.
+ * hbl_gemm_codes use: 0 = by size (default: for M >= 128 tokens the tcgen05
+ * tensor-core kernel with one 128 x 256 tile per CTA; for 9..64 tokens the
+ * decode kernel split over K across a thread-block cluster (K >= 512); for
+ * 1..8 tokens the decode kernel with one CTA per 16 rows; the warp-level
+ * split-K kernel otherwise), 1 = always the warp-level split-K kernel,
+ * 2 = always the persistent tcgen05 kernel (128 x 128 tiles), 3 = as 0 but
+ * never the cluster or streaming decode kernels, 4 = always the one-tile
+ * tcgen05 kernel, 5 = as 0 (the weight-streaming decode kernel is the default
+ * for 1..16 tokens with K % 2048 == 0).
+ * All give identical results; the knob exists to check and time each one.
+ * Process-wide.
  */
 int hbl_set_gemm_path(int path);
 
