@@ -298,6 +298,22 @@ def secondary(torch, hbl, layer, inputs):
             "us_per_forward": ms * 1e3, "tokens_per_s": case.M / (ms * 1e-3),
             "weight_GBps": case.N * case.K / 4 / (ms * 1e-3) / 1e9}
         del g, Wpks
+    # a large decode shape: 64 MiB of packed weights per forward (16 weight sets, 1 GiB per step)
+    big = inputs.sweep_case(16, 16384, 16384, 4, 1)
+    c = dict(M=big.M, K=big.K, N=big.N, act_bits=big.act_bits, use_hadamard=big.use_hadamard)
+    X = big.make_x().cuda()
+    Wpk, wsc = layer.pack_weights(big.make_w().cuda())
+    Wpks = [Wpk] + [Wpk.clone() for _ in range(15)]
+    Y = torch.empty(big.M, big.N, dtype=torch.bfloat16, device="cuda")
+    ws = layer.workspace(big.M, big.K, big.N, "cuda")
+    hbl.hbl_forward_ws(X, big.M, big.K, big.N, Wpk, wsc, 4, 1, Y, ws, ws.numel())
+    g = capture_step(torch, hbl, X, Wpks, wsc, Y, ws, c)
+    ms = timed_replays(torch, None, g, 3, 10, 1) / (10 * len(Wpks))
+    out["decode M=16 K=16384 N=16384 a4"] = {
+        "us_per_forward": ms * 1e3, "tokens_per_s": big.M / (ms * 1e-3),
+        "weight_GBps": big.N * big.K / 4 / (ms * 1e-3) / 1e9}
+    del g, Wpks
+    torch.cuda.empty_cache()
     case = inputs.prefill_down_case()
     X = case.make_x().cuda()
     Wpk, wsc = layer.pack_weights(case.make_w().cuda())
@@ -415,6 +431,8 @@ def profile_case(which: str):
         case = inputs.prefill_down_case()
     elif which == "decode":
         case = [c for c in inputs.decode_oproj_cases((HEAD["M"],), (HEAD["act_bits"],))][0]
+    elif which == "decode_big":
+        case = inputs.sweep_case(16, 16384, 16384, 4, 1)
     else:
         raise SystemExit(f"unknown profile case {which}")
     X = case.make_x().cuda()
@@ -436,7 +454,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile-case", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "decode_big"], default=None,
                     help="run one short fixed case (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile_case:

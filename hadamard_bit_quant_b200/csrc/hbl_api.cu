@@ -891,6 +891,16 @@ int hbl_profile_get(int i, char* name, int name_len, int* launches, double* tota
   return HBL_OK;
 }
 
+int hbl_selftest_wait_timeout(int timeout_us, int* gave_up, hbl_stream stream) {
+  if (timeout_us < 1 || timeout_us > 10000000) return HBL_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  int st = ensure_device(&d);
+  if (st) return st;
+  wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)timeout_us * 1000ull, gave_up);
+  return launch_status();
+}
+
 int hbl_get_device_error(hbl_stream stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return HBL_ERR_CUDA;

@@ -21,6 +21,40 @@ __device__ unsigned int g_error_word = 0;
 
 HBL_DEVINL void set_device_error(unsigned int code) { atomicOr(&g_error_word, 1u << code); }
 
+HBL_DEVINL unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+// Failure-detection check: an mbarrier that nothing will ever complete, waited
+// on with the same bounded try_wait loop the pipelined kernels use, but with a
+// limit of `timeout_ns`. On expiry the kernel records HBL_ERR_TIMEOUT in the
+// device error word and returns normally.
+__global__ void wait_timeout_selftest_kernel(unsigned long long timeout_ns, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(&bar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;\n" ::"r"(a) : "memory");   // needs 2 arrivals
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(a) : "memory");   // only 1 ever comes
+  }
+  __syncthreads();
+  const unsigned long long t0 = global_ns();
+  uint32_t ok = 0;
+  while (true) {
+    asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\nselp.u32 %0, 1, 0, p;\n}\n"
+                 : "=r"(ok)
+                 : "r"(a)
+                 : "memory");
+    if (ok) break;
+    if (global_ns() - t0 > timeout_ns) break;
+  }
+  if (!ok && threadIdx.x == 0) {
+    set_device_error(HBL_ERR_TIMEOUT);
+    if (gave_up) *gave_up = 1;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Packed weight layout (opaque to callers).
 //

@@ -36,6 +36,7 @@ SIGNATURES = [
     ("hbl_pack_weights_rotated", _I, [_P, _I, _I, _P, _P, _P, _P]),
     ("hbl_hadamard_backward_f32", _I, [_P, _I, _I, _P, _P]),
     ("hbl_quantize_qkv", _I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    ("hbl_selftest_wait_timeout", _I, [_I, _P, _P]),
     ("hbl_get_device_error", _I, [_P]),
     ("hbl_set_gemm_path", _I, [_I]),
     ("hbl_profile_enable", _I, [_I]),
@@ -167,6 +168,11 @@ def hbl_hadamard_backward_f32(dXr, M, K, dX, stream=None):
 def hbl_quantize_qkv(X, T, H, d, bits, bos_token, codes, gamma, stream=None):
     return _check(lib().hbl_quantize_qkv(_ptr(X), T, H, d, bits, bos_token, _ptr(codes), _ptr(gamma),
                                          _stream(stream)), "hbl_quantize_qkv")
+
+
+def hbl_selftest_wait_timeout(timeout_us, gave_up=None, stream=None):
+    return _check(lib().hbl_selftest_wait_timeout(int(timeout_us), _ptr(gave_up), _stream(stream)),
+                  "hbl_selftest_wait_timeout")
 
 
 def hbl_get_device_error(stream=None):

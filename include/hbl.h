@@ -181,7 +181,10 @@ int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard
  * hbl_gemm_codes -- acc[m, n] = sum_k codes[m, k] * T[n, k], exactly, in int32.
  *   codes : device int8 M x K (any values in [-128, 127]).
  *   acc   : device int32 M x N.
- * Same shape rules as hbl_forward_ws (K % 256 == 0).
+ * Same shape rules as hbl_forward_ws (K % 256 == 0). The per-token code
+ * sums go to a small library-owned scratch that grows on demand (a
+ * cudaMalloc), shared with hbl_forward: make a first call of each size
+ * before any stream capture, and do not overlap calls on different streams.
  */
 int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
                    int32_t* acc, hbl_stream stream);
@@ -266,6 +269,18 @@ int hbl_get_device_error(hbl_stream stream);
  * Process-wide.
  */
 int hbl_set_gemm_path(int path);
+
+/*
+ * hbl_selftest_wait_timeout -- failure-detection check of the bounded waits.
+ * Launches one CTA whose mbarrier wait can never complete (the barrier
+ * expects two arrivals and gets one). The wait is the same bounded try_wait
+ * loop the pipelined kernels use, here limited to timeout_us microseconds
+ * (1 .. 10^7). On expiry the kernel records HBL_ERR_TIMEOUT in the device
+ * error word, writes 1 to *gave_up (device int, may be NULL) and exits
+ * normally: no trap, no hang, the context stays usable. The next
+ * hbl_get_device_error returns HBL_ERR_TIMEOUT.
+ */
+int hbl_selftest_wait_timeout(int timeout_us, int* gave_up, hbl_stream stream);
 
 /* ------------------------------------------------------------------------
  * Per-kernel timing of the library's own launches.
