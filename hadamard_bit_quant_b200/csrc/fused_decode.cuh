@@ -1,0 +1,567 @@
+// Fused decode forward: online Hadamard, per-token quantiser, ternary x int8
+// GEMM and dequant epilogue in ONE kernel, for 1..16 tokens.
+//
+// BitNet v2 architecture walkthrough, section 3.4 "H-BitLinear: The Composite
+// Layer", Eq. 9 (with Eq. 3-6 for the transform, Eq. 7 / Eq. 8 for the
+// quantiser): Y = dequant( Q_A( H x ) (x) T ).
+//
+// With a few tokens the forward is a pass over N*K/4 bytes of packed weights
+// plus a chain of short dependent steps (transform, statistic, codes, MMA,
+// epilogue). Two kernels cost two grid boundaries and an L2 round trip of the
+// codes; this kernel keeps every intermediate on chip:
+//   * one CTA per SM, grouped into clusters of CS CTAs (CS = 1, 2, 4 or 8);
+//   * a producer warp streams the weights of the CTA's 16-row groups through
+//     a TMA ring from the first instruction on, before the kernel waits for
+//     the grid that produced X (programmatic dependent launch);
+//   * the 8 consumer warps of cluster rank r transform and quantise token rows
+//     r, r + CS, ... (two rows at a time, 256 threads per row, E = K/256
+//     values per thread, butterflies in registers, passes exchanged through
+//     padded shared memory), then write each row's codes, its scale and its
+//     per-warp code sums into the shared memory of EVERY CTA of the cluster
+//     (distributed shared memory). After a cluster barrier each CTA holds all
+//     M x K codes;
+//   * the consumers then run the m16n8k32 MMAs of their groups (weights as A,
+//     u = t + 1 unpacked in registers; codes as B), batches of groups
+//     interleaved for independent accumulator chains, add the 8 warps' partial
+//     sums in shared memory, subtract the code sums and store bf16.
+// Every mbarrier wait is bounded; a CTA that gives up sets the device error
+// word, still takes part in both cluster barriers, and writes no output.
+#pragma once
+#include <cuda.h>
+#include "hbl_common.cuh"
+#include "fwht_quant.cuh"
+#include "gemm_mma.cuh"
+
+namespace hbl {
+namespace fdec {
+
+constexpr int kGroupRows = 16;
+constexpr int kChunk = 2048;
+constexpr int kConsumers = 8;
+constexpr int kRowThreads = 32 * kConsumers;        // threads per token row
+constexpr int kThreads = 32 * (kConsumers + 1);
+constexpr int kStages = 8;
+constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB = 4 boxes of [16][128 B]
+constexpr int kMaxGroups = 8;
+constexpr int kBatch = 4;
+constexpr int kRowBatch = 2;                        // token rows transformed together
+constexpr int kMaxTokens = 16;
+constexpr long long kSpinLimit = 4000000000ll;
+
+__host__ __device__ constexpr int ilog2_c(int x) { return x <= 1 ? 0 : 1 + ilog2_c(x / 2); }
+
+HBL_DEVINL uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+HBL_DEVINL void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(su32(b)), "r"(count) : "memory");
+}
+HBL_DEVINL void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+HBL_DEVINL void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(su32(b)) : "memory");
+}
+HBL_DEVINL bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+HBL_DEVINL bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(b, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > kSpinLimit) {
+      *abort = 1;
+      set_device_error(HBL_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+HBL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
+          su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+HBL_DEVINL uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+HBL_DEVINL uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
+  return r;
+}
+HBL_DEVINL uint32_t map_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+HBL_DEVINL void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+HBL_DEVINL void st_cluster_v2(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};\n" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+HBL_DEVINL void st_cluster_u32(uint32_t addr, uint32_t a) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(a) : "memory");
+}
+HBL_DEVINL void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory"); }
+HBL_DEVINL void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
+HBL_DEVINL void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
+// Named barrier over the consumer warps only (the producer never joins it).
+HBL_DEVINL void consumers_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(kRowThreads) : "memory"); }
+
+template <int LOG_K, int MT>
+struct Layout {
+  static constexpr int K = 1 << LOG_K;
+  static constexpr int E = K / kRowThreads;
+  static constexpr int KPAD = K + K / E;
+  static constexpr size_t kRing = (size_t)kStages * kUnitBytes;
+  static constexpr size_t kCodes = (size_t)MT * K;           // K/128 boxes of [MT][128 B]
+  static constexpr size_t kX = (size_t)kRowBatch * KPAD * 4;
+  static constexpr size_t oCodes = kRing;
+  static constexpr size_t oX = oCodes + kCodes;
+  static constexpr size_t oScale = oX + kX;                   // float [kMaxTokens]
+  static constexpr size_t oCsum = oScale + kMaxTokens * 4;    // int [kMaxTokens][kConsumers]
+  static constexpr size_t oRed = oCsum + kMaxTokens * kConsumers * 4;   // float [kRowBatch * 2][kConsumers]
+  static constexpr size_t oBars = oRed + kRowBatch * 2 * kConsumers * 4;
+  static constexpr size_t kBytes = 1024 + oBars + 2 * kStages * 8 + 16;
+  static_assert(kMaxGroups * kConsumers * kGroupRows * MT * 4 <= kRing, "reduction must fit in the ring");
+};
+
+// Byte offset of the 16-byte code chunk holding k = 16*c16 .. 16*c16+15 of
+// token m: box k/128 of [MT][128 B], 128B-swizzled by m % 8 (the layout a
+// TMA SWIZZLE_128B load of a [MT][128] box produces).
+template <int MT>
+HBL_DEVINL uint32_t code_off(int m, int c16) {
+  return (uint32_t)((c16 >> 3) * (MT * 128) + m * 128 + (((c16 & 7) ^ (m & 7)) << 4));
+}
+
+// Sum (or max) over the 256 consumer threads of NR values at once (one
+// barrier for all rows). Per row: butterfly within each warp, then warps
+// 0..7 in order (the order of the quantiser kernels).
+template <int NR, bool IS_MAX>
+HBL_DEVINL void rows_reduce_n(float (&x)[NR], float* slot) {
+#pragma unroll
+  for (int r = 0; r < NR; ++r)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[r], off);
+      x[r] = IS_MAX ? fmaxf(x[r], o) : x[r] + o;
+    }
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int r = 0; r < NR; ++r) slot[r * kConsumers + (threadIdx.x >> 5)] = x[r];
+  }
+  consumers_sync();
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    float a = slot[r * kConsumers];
+#pragma unroll
+    for (int i = 1; i < kConsumers; ++i) a = IS_MAX ? fmaxf(a, slot[r * kConsumers + i]) : a + slot[r * kConsumers + i];
+    x[r] = a;
+  }
+}
+
+// Phase 1 for NR (1 or 2) token rows m0, m0 + cs: load, optional RMSNorm,
+// optional transform, quantise, and write codes, scale and per-warp code sums
+// into the shared memory of every CTA of the cluster (of this CTA alone when
+// cs == 1). `cw1` is true until this CTA has waited on cluster barrier #1,
+// which must precede the first remote store.
+template <int LOG_K, int MT, int NR>
+HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, uint32_t cs, bool had, bool int8, bool ln,
+                           const float* __restrict__ gain, float* xb, float* s_red, uint8_t* cbuf, float* s_scale,
+                           int* s_csum, bool& cw1) {
+  constexpr int K = 1 << LOG_K, E = K / kRowThreads, G = ilog2_c(E), P = (LOG_K + G - 1) / G, KPAD = K + K / E;
+  constexpr int T = kRowThreads;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  float v[NR][E];
+  float nrm[NR];
+  // loads: the flag branches stay outside the unrolled loops so that every
+  // load of a row is in flight at once
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    const uint16_t* xr = X + (size_t)(m0 + r * (int)cs) * K;
+    nrm[r] = 1.f;
+    if (had) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) v[r][j] = bf16_bits_to_float(__ldg(xr + t + j * T));
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(xr + (size_t)E * t);
+      uint4 w4[E / 8];
+#pragma unroll
+      for (int q = 0; q < E / 8; ++q) w4[q] = __ldg(src + q);
+#pragma unroll
+      for (int q = 0; q < E / 8; ++q) {
+        const uint32_t w[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[r][8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+          v[r][8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+      }
+    }
+  }
+  if (ln) {
+    // RMSNorm: sum of squares of the raw row; the gain per channel (on the
+    // pass-0 layout with the transform, on the final layout without); the
+    // per-token factor folded into the transform's scale, or applied.
+    float tot[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      float ssq = 0.f;
+#pragma unroll
+      for (int j = 0; j < E; ++j) ssq = __fmaf_rn(v[r][j], v[r][j], ssq);
+      tot[r] = ssq;
+    }
+    consumers_sync();   // the slots' previous readers are done
+    rows_reduce_n<NR, false>(tot, s_red);
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const float rr = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot[r], (float)K), kRmsEps)));
+      if (had) {
+        if (gain) {
+#pragma unroll
+          for (int j = 0; j < E; ++j) v[r][j] = __fmul_rn(v[r][j], __ldg(gain + t + j * T));
+        }
+        nrm[r] = rr;
+      } else if (gain) {
+#pragma unroll
+        for (int j = 0; j < E; ++j) v[r][j] = __fmul_rn(__fmul_rn(v[r][j], __ldg(gain + E * t + j)), rr);
+      } else {
+#pragma unroll
+        for (int j = 0; j < E; ++j) v[r][j] = __fmul_rn(__fmul_rn(v[r][j], 1.f), rr);
+      }
+    }
+  }
+  if (had) {
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+      const int hi = LOG_K - p * G;
+      const int lo = hi - G > 0 ? hi - G : 0;
+      if (p > 0) {
+        const int hi_prev = LOG_K - (p - 1) * G;
+        const int lo_prev = hi_prev - G > 0 ? hi_prev - G : 0;
+        consumers_sync();   // the previous readers of xb are done
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+          for (int j = 0; j < E; ++j) xb[r * KPAD + pad<G>(pass_index<G>(t, j, lo_prev))] = v[r][j];
+        consumers_sync();
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+#pragma unroll
+          for (int j = 0; j < E; ++j) v[r][j] = xb[r * KPAD + pad<G>(pass_index<G>(t, j, lo))];
+      }
+#pragma unroll
+      for (int r = 0; r < NR; ++r) butterflies<E>(v[r], hi - lo);
+    }
+    float sc = __uint_as_float((uint32_t)(127 - LOG_K / 2) << 23);
+    if (LOG_K & 1) sc *= 0.70710678118654752f;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) nrm[r] = __fmul_rn(sc, nrm[r]);
+  }
+  // thread t now holds elements E*t .. E*t+E-1 of each row: the statistic
+  float stat[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    float part = 0.f;
+    if (!int8) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) part += fabsf(v[r][j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < E; ++j) part = fmaxf(part, fabsf(v[r][j]));
+    }
+    stat[r] = part;
+  }
+  consumers_sync();   // the slots' previous readers are done
+  if (int8) rows_reduce_n<NR, true>(stat, s_red + 2 * kConsumers);
+  else rows_reduce_n<NR, false>(stat, s_red + 2 * kConsumers);
+  if (cw1) {
+    cluster_wait();   // #1: every peer runs, so its shared memory may be written
+    cw1 = false;
+  }
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    const int m = m0 + r * (int)cs;
+    const float rs = __fmul_rn(stat[r], nrm[r]);
+    float mult, scale;
+    int lo, hi;
+    if (!int8) {
+      const float beta = __fdiv_rn(rs, (float)K);
+      mult = __fdiv_rn(kSqrt7, __fadd_rn(beta, kEps));
+      scale = __fdiv_rn(beta, kSqrt7);
+      lo = -8; hi = 7;
+    } else {
+      mult = __fdiv_rn(127.f, __fadd_rn(rs, kEps));
+      scale = __fdiv_rn(rs, 127.f);
+      lo = -128; hi = 127;
+    }
+    mult = __fmul_rn(mult, nrm[r]);
+    int csum = 0;
+    uint32_t packed[E / 4];
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) {
+      uint32_t w = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = clampi(__float2int_rn(__fmul_rn(mult, v[r][4 * q + i])), lo, hi);
+        csum += c;
+        w |= ((uint32_t)(c & 0xff)) << (8 * i);
+      }
+      packed[q] = w;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) csum += __shfl_xor_sync(0xffffffffu, csum, off);
+    if (cs == 1) {
+      if constexpr (E == 8) {
+        *reinterpret_cast<uint2*>(cbuf + code_off<MT>(m, t >> 1) + ((t & 1) << 3)) = make_uint2(packed[0], packed[1]);
+      } else {
+#pragma unroll
+        for (int h = 0; h < E / 16; ++h)
+          *reinterpret_cast<uint4*>(cbuf + code_off<MT>(m, t * (E / 16) + h)) =
+              make_uint4(packed[4 * h], packed[4 * h + 1], packed[4 * h + 2], packed[4 * h + 3]);
+      }
+      if (lane == 0) s_csum[m * kConsumers + warp] = csum;
+      if (t == 0) s_scale[m] = scale;
+    } else {
+      const uint32_t scale_bits = __float_as_uint(scale);
+      for (uint32_t q = 0; q < cs; ++q) {
+        if constexpr (E == 8) {
+          const uint32_t off = code_off<MT>(m, t >> 1) + ((t & 1) << 3);
+          st_cluster_v2(map_rank(su32(cbuf + off), q), packed[0], packed[1]);
+        } else {
+#pragma unroll
+          for (int h = 0; h < E / 16; ++h) {
+            const uint32_t off = code_off<MT>(m, t * (E / 16) + h);
+            st_cluster_v4(map_rank(su32(cbuf + off), q), packed[4 * h], packed[4 * h + 1], packed[4 * h + 2],
+                          packed[4 * h + 3]);
+          }
+        }
+        if (lane == 0) st_cluster_u32(map_rank(su32(s_csum + m * kConsumers + warp), q), (uint32_t)csum);
+        if (t == 0) st_cluster_u32(map_rank(su32(s_scale + m), q), scale_bits);
+      }
+    }
+  }
+}
+
+// flags: bit 0 use_hadamard, bit 1 INT8 (else INT4), bit 2 RMSNorm prologue.
+template <int LOG_K, int TN>
+__global__ void __launch_bounds__(kThreads, 1)
+fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* __restrict__ X, int M, int N,
+                    const float* __restrict__ gain, const float* __restrict__ alpha, int flags,
+                    uint16_t* __restrict__ Y) {
+  constexpr int MT = 8 * TN;
+  using Lay = Layout<LOG_K, MT>;
+  constexpr int nchunks = Lay::K / kChunk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = base;
+  uint8_t* cbuf = base + Lay::oCodes;
+  float* xb = reinterpret_cast<float*>(base + Lay::oX);
+  float* s_scale = reinterpret_cast<float*>(base + Lay::oScale);
+  int* s_csum = reinterpret_cast<int*>(base + Lay::oCsum);
+  float* s_red = reinterpret_cast<float*>(base + Lay::oRed);
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(base + Lay::oBars);
+  uint64_t* wempty = wfull + kStages;
+  volatile int* abort = reinterpret_cast<volatile int*>(wempty + kStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_rank(), csize = cluster_size();
+  const int groups = N / kGroupRows;
+  const int Gd = gridDim.x;
+  const int ng = (groups - (int)blockIdx.x + Gd - 1) / Gd;
+  const int units = nchunks * ng;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], kConsumers);
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+  if (csize > 1) cluster_arrive_relaxed();   // #1: this CTA runs (peers may write its shared memory after #1)
+
+  if (warp == kConsumers) {
+    // ----- producer: the weight ring (independent of the previous grid) -----
+    int u = 0;
+    auto issue_w = [&](int uu) {
+      const int s = uu % kStages;
+      const int c = uu / ng, gl = uu % ng;
+      const int row0 = ((int)blockIdx.x + gl * Gd) * kGroupRows;
+      mbar_expect_tx(&wfull[s], kUnitBytes);
+      uint8_t* dst = ring + (size_t)s * kUnitBytes;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) tma_load_2d(dst + b * (kGroupRows * 128), &map_w, &wfull[s], c * (kChunk / 4) + b * 128, row0);
+    };
+    if (lane == 0)
+      for (; u < units && u < kStages; ++u) issue_w(u);
+    __syncwarp();
+    if (csize > 1) {
+      cluster_wait();             // #1
+      cluster_arrive_relaxed();   // #2: the producer writes nothing a peer reads
+    }
+    if (lane == 0) {
+      bool ok = true;
+      for (; u < units && ok; ++u) {
+        const int s = u % kStages;
+        if (!mbar_wait(&wempty[s], (uint32_t)((u / kStages) - 1) & 1u, abort)) { ok = false; break; }
+        issue_w(u);
+      }
+      // bounded drain of the copies issued last
+      for (int q = (u > kStages ? u - kStages : 0); q < u; ++q) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&wfull[q % kStages], (uint32_t)(q / kStages) & 1u) && clock64() - t0 < kSpinLimit) {
+        }
+      }
+    }
+    __syncwarp();
+    if (csize > 1) cluster_wait();   // #2
+  } else {
+    // ----- consumers, phase 1: transform + quantise this CTA's token rows -----
+    const bool had = (flags & 1) != 0, int8 = (flags & 2) != 0, ln = (flags & 4) != 0;
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");   // X is ready past this point
+    const float a_w = __ldg(alpha);
+    bool cw1 = csize > 1;
+    for (int m0 = (int)crank; m0 < M; m0 += (int)csize * kRowBatch) {
+      if (m0 + (int)csize < M)
+        rows_phase<LOG_K, MT, 2>(X, m0, csize, had, int8, ln, gain, xb, s_red, cbuf, s_scale, s_csum, cw1);
+      else
+        rows_phase<LOG_K, MT, 1>(X, m0, csize, had, int8, ln, gain, xb, s_red, cbuf, s_scale, s_csum, cw1);
+    }
+    if (csize > 1) {
+      if (cw1) cluster_wait();   // #1 (this CTA had no rows)
+      cluster_arrive_release();  // #2: this CTA's writes into the cluster are done
+      cluster_wait();            // #2: every row of codes is here
+    } else {
+      consumers_sync();          // every row of codes is here
+    }
+
+    // ----- consumers, phase 2: MMAs over the weight ring -----
+    const int g = lane >> 2, tig = lane & 3;
+    constexpr int SPLIT = TN == 1 ? 2 : 1;
+    int acc[kMaxGroups][TN * SPLIT][4];
+#pragma unroll
+    for (int a = 0; a < kMaxGroups; ++a)
+#pragma unroll
+      for (int i = 0; i < TN * SPLIT; ++i)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
+    bool ok = true;
+    const int ch = ((warp & 1) << 2) + tig;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      uint2 bf[TN][8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int box = c * (kChunk / 128) + 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
+#pragma unroll
+        for (int i = 0; i < TN; ++i) {
+          const int m = 8 * i + g;
+          bf[i][q] = *reinterpret_cast<const uint2*>(cbuf + box * (MT * 128) + m * 128 + ((cch ^ (m & 7)) << 4) +
+                                                     ((tig & 1) << 3));
+        }
+      }
+#pragma unroll
+      for (int gb = 0; gb < kMaxGroups; gb += kBatch) {
+        if (gb < ng && ok) {
+          uint32_t A4[kBatch][4], B4[kBatch][4];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            if (gb + b < ng) {
+              const int u = c * ng + gb + b;
+              const int s = u % kStages;
+              if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
+              const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
+              const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
+              const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+              A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
+              B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+              if (gb + b < ng) mbar_arrive(&wempty[(c * ng + gb + b) % kStages]);
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int w = q >> 1, jj = 2 * (q & 1);
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+              if (gb + b < ng) {
+                const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj),
+                                       unpack_u8x4(A4[b][w], jj + 1), unpack_u8x4(B4[b][w], jj + 1)};
+#pragma unroll
+                for (int i = 0; i < TN; ++i)
+                  mma_u8s8_16832(acc[gb + b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
+              }
+            }
+          }
+        }
+      }
+    }
+    if constexpr (SPLIT == 2) {
+#pragma unroll
+      for (int a = 0; a < kMaxGroups; ++a)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
+    }
+    // partial sums of the 8 warps -> shared memory, aliasing the ring once
+    // every consumer is past its last unit: red[warp][group][row][token]
+    consumers_sync();
+    if (ok && *abort == 0) {
+      int* red = reinterpret_cast<int*>(ring);
+#pragma unroll
+      for (int gl = 0; gl < kMaxGroups; ++gl) {
+        if (gl < ng) {
+#pragma unroll
+          for (int i = 0; i < TN; ++i)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int row = g + ((r >> 1) << 3);
+              const int tok = 8 * i + 2 * tig + (r & 1);
+              red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
+            }
+        }
+      }
+    }
+    consumers_sync();
+    if (ok && *abort == 0) {
+      const int* red = reinterpret_cast<const int*>(ring);
+      const int per_group = kGroupRows * MT;
+      for (int e = threadIdx.x; e < ng * per_group; e += kRowThreads) {
+        const int gl = e / per_group, rem = e % per_group;
+        const int tok = rem / kGroupRows, row = rem % kGroupRows;
+        const int n = ((int)blockIdx.x + gl * Gd) * kGroupRows + row;
+        if (tok < M) {
+          int s = 0;
+#pragma unroll
+          for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * kGroupRows + row) * MT + tok];
+          int cs = 0;
+#pragma unroll
+          for (int w = 0; w < kConsumers; ++w) cs += s_csum[tok * kConsumers + w];
+          s -= cs;
+          const float y = __fmul_rn(__fmul_rn((float)s, s_scale[tok]), a_w);
+          Y[(size_t)tok * N + n] = float_to_bf16_bits(y);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace fdec
+}  // namespace hbl

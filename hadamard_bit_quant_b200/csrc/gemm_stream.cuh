@@ -42,6 +42,7 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = HBL_STREAM_STAGES;
 constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB: 4 boxes of [16][128 B]
 constexpr int kMaxGroups = 8;                      // per CTA
+constexpr int kBatch = 4;                          // groups whose MMAs are interleaved
 constexpr long long kSpinLimit = 4000000000ll;
 
 HBL_DEVINL uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -188,13 +189,17 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   } else {
     // ----- consumers: warp w takes 256-k block w of every unit -----
+    // The MMAs of up to kBatch groups are interleaved q by q so that
+    // 2 * kBatch independent accumulator chains are in flight (with one token
+    // tile, even and odd q accumulate separately and are added at the end).
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     const int g = lane >> 2, tig = lane & 3;
-    int acc[kMaxGroups][TN][4];
+    constexpr int SPLIT = TN == 1 ? 2 : 1;
+    int acc[kMaxGroups][TN * SPLIT][4];
 #pragma unroll
     for (int a = 0; a < kMaxGroups; ++a)
 #pragma unroll
-      for (int i = 0; i < TN; ++i)
+      for (int i = 0; i < TN * SPLIT; ++i)
 #pragma unroll
         for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
     bool ok = true;
@@ -215,30 +220,53 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
+      const int ch = ((warp & 1) << 2) + tig;
 #pragma unroll
-      for (int gl = 0; gl < kMaxGroups; ++gl) {
-        if (gl < ng) {
-          const int u = c * ng + gl;
-          const int s = u % kStages;
-          if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) { ok = false; break; }
-          const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
-          const int ch = ((warp & 1) << 2) + tig;
-          const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
-          const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+      for (int gb = 0; gb < kMaxGroups; gb += kBatch) {
+        if (gb < ng && ok) {
+          uint32_t A4[kBatch][4], B4[kBatch][4];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            if (gb + b < ng) {
+              const int u = c * ng + gb + b;
+              const int s = u % kStages;
+              if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
+              const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
+              const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
+              const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+              A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
+              B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
+            }
+          }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&wempty[s]);
-          const uint32_t A4[4] = {pa.x, pa.y, pa.z, pa.w};
-          const uint32_t B4[4] = {pb.x, pb.y, pb.z, pb.w};
+          if (lane == 0) {
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+              if (gb + b < ng) mbar_arrive(&wempty[(c * ng + gb + b) % kStages]);
+          }
+          if (!ok) break;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int w = q >> 1, jj = 2 * (q & 1);
-            const uint32_t a[4] = {unpack_u8x4(A4[w], jj), unpack_u8x4(B4[w], jj), unpack_u8x4(A4[w], jj + 1),
-                                   unpack_u8x4(B4[w], jj + 1)};
 #pragma unroll
-            for (int i = 0; i < TN; ++i) mma_u8s8_16832(acc[gl][i], a, bf[i][q].x, bf[i][q].y);
+            for (int b = 0; b < kBatch; ++b) {
+              if (gb + b < ng) {
+                const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj),
+                                       unpack_u8x4(A4[b][w], jj + 1), unpack_u8x4(B4[b][w], jj + 1)};
+#pragma unroll
+                for (int i = 0; i < TN; ++i)
+                  mma_u8s8_16832(acc[gb + b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
+              }
+            }
           }
         }
       }
+    }
+    if constexpr (SPLIT == 2) {
+#pragma unroll
+      for (int a = 0; a < kMaxGroups; ++a)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
     }
     // partial sums of the 8 warps -> shared memory (aliases the ring, so only
     // after every warp is done with it): red[warp][group][row][token]

@@ -18,6 +18,7 @@
 #include "gemm_decode.cuh"
 #include "gemm_decode2.cuh"
 #include "gemm_stream.cuh"
+#include "fused_decode.cuh"
 #include "qkv_quant.cuh"
 
 namespace hbl {
@@ -245,20 +246,19 @@ void launch_fwht(const FwhtArgs& a, cudaStream_t s) {
 }
 
 constexpr int kLatencyTokens = 64;
-#ifndef HBL_FWHT_LAT_G12
-#define HBL_FWHT_LAT_G12 3
-#endif
 
-// Few tokens: more threads per token (8 or 16 values each) for latency; many
-// tokens: 32-128 values per thread for throughput.
+// Few tokens: more threads per token for latency; many tokens: 32-128 values
+// per thread for throughput. For K = 2048, 4096 and 8192 the few-token
+// configuration is 256 threads per token (E = K/256), the same split and
+// summation order as the fused decode kernel, so both produce the same bits.
 template <int MODE, bool IN_F32 = false, bool LN = false>
 int dispatch_fwht(const FwhtArgs& a, int K, cudaStream_t s) {
   if (a.M <= kLatencyTokens) {
     switch (ilog2(K)) {
       case 10: launch_fwht<10, 3, MODE, IN_F32, LN>(a, s); return launch_status();
       case 11: launch_fwht<11, 3, MODE, IN_F32, LN>(a, s); return launch_status();
-      case 12: launch_fwht<12, HBL_FWHT_LAT_G12, MODE, IN_F32, LN>(a, s); return launch_status();
-      case 13: launch_fwht<13, 3, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 12: launch_fwht<12, 4, MODE, IN_F32, LN>(a, s); return launch_status();
+      case 13: launch_fwht<13, 5, MODE, IN_F32, LN>(a, s); return launch_status();
       case 14: launch_fwht<14, 4, MODE, IN_F32, LN>(a, s); return launch_status();
       default: break;
     }
@@ -282,8 +282,15 @@ int dispatch_rows(const uint16_t* X, int M, int K, const float* gain, int8_t* co
                   int32_t* csum, cudaStream_t s) {
   auto blocks = [](int T) { return (T + 31) / 32 * 32; };
   ProfScope ps("quant_rows", s);
-  if (K <= 8192)
+  // K = 2048, 4096, 8192: 256 threads with K/256 values each, the split of the fused decode kernel
+  if (K <= 2048)
     launch_pdl(quant_rows_kernel<8, MODE, LN>, dim3(M), dim3(blocks(K / 8)), 0, s, X, M, K, gain, codes, scales,
+               csum);
+  else if (K <= 4096)
+    launch_pdl(quant_rows_kernel<16, MODE, LN>, dim3(M), dim3(blocks(K / 16)), 0, s, X, M, K, gain, codes, scales,
+               csum);
+  else if (K <= 8192)
+    launch_pdl(quant_rows_kernel<32, MODE, LN>, dim3(M), dim3(blocks(K / 32)), 0, s, X, M, K, gain, codes, scales,
                csum);
   else if (K <= 16384)
     launch_pdl(quant_rows_kernel<16, MODE, LN>, dim3(M), dim3(blocks(K / 16)), 0, s, X, M, K, gain, codes, scales,
@@ -384,7 +391,8 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 
 // 0 auto, 1 warp-level mma.sync, 2 tcgen05 persistent (128 x 128 tiles), 3 decode without
 // clusters or streaming, 4 tcgen05 one 128 x 256 tile per CTA (the default for M >= 128),
-// 5 weight-streaming decode (the default for M <= 16 where it fits)
+// 5 weight-streaming decode (the default for M <= 16 where it fits), 6 as 0 (the forward
+// takes the fused single-kernel decode wherever it fits; 0 does the same)
 int g_gemm_path = 0;
 
 bool use_tc_path(int M) {
@@ -580,6 +588,88 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
   return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Fused single-kernel decode forward (1..16 tokens, K in {2048, 4096, 8192}).
+// ---------------------------------------------------------------------------
+constexpr int kFusedNotApplicable = -1;
+
+int fused_cluster_size(int M) { return M <= 2 ? 1 : (M <= 4 ? 2 : (M <= 8 ? 4 : 8)); }
+
+template <int LOG_K, int TN>
+int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const float* gain, const float* alpha,
+                 int flags, uint16_t* Y, int sm_count, cudaStream_t s) {
+  auto* kern = fdec::fused_decode_kernel<LOG_K, TN>;
+  const size_t smem = fdec::Layout<LOG_K, 8 * TN>::kBytes;
+  ensure_smem_attr(kern, smem);
+  const int CS = fused_cluster_size(M);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(fdec::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = kUsePdl ? 2 : 1;
+  // clusters that fit at once (cached per device, kernel and cluster size)
+  struct Entry { int dev; const void* fn; int cs; int clusters; };
+  static std::mutex mu;
+  static std::vector<Entry> known;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int clusters = -1;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (auto& e : known)
+      if (e.dev == dev && e.fn == (const void*)kern && e.cs == CS) clusters = e.clusters;
+    if (clusters < 0) {
+      cfg.gridDim = dim3((unsigned)(sm_count / CS * CS));
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        clusters = 0;
+      }
+      known.push_back(Entry{dev, (const void*)kern, CS, clusters});
+    }
+  }
+  int grid = clusters * CS;
+  if (grid > sm_count / CS * CS) grid = sm_count / CS * CS;
+  const int groups = N / fdec::kGroupRows;
+  if (grid < CS || groups > fdec::kMaxGroups * grid) return kFusedNotApplicable;
+  cfg.gridDim = dim3((unsigned)grid);
+  ProfScope ps("fused_decode", s);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, X, M, N, gain, alpha, flags, Y);
+  return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
+}
+
+bool fused_fits(int M, int K, int N) {
+  if (M < 1 || M > fdec::kMaxTokens || N % fdec::kGroupRows != 0) return false;
+  if (K != 2048 && K != 4096 && K != 8192) return false;
+  const int MT = M <= 8 ? 8 : 16;
+  return (long long)MT * K <= 65536;
+}
+
+int run_fused_decode(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale, int act_bits,
+                     int use_hadamard, bool ln, const float* gain, uint16_t* Y, int sm_count, cudaStream_t s) {
+  CUtensorMap mw;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, fdec::kGroupRows, true))
+    return HBL_ERR_CUDA;
+  const int flags = (use_hadamard ? 1 : 0) | (act_bits == 8 ? 2 : 0) | (ln ? 4 : 0);
+  const bool tn1 = M <= 8;
+  switch (K) {
+    case 2048: return tn1 ? launch_fused<11, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
+                          : launch_fused<11, 2>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s);
+    case 4096: return tn1 ? launch_fused<12, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
+                          : launch_fused<12, 2>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s);
+    case 8192: return tn1 ? launch_fused<13, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
+                          : kFusedNotApplicable;
+    default: return kFusedNotApplicable;
+  }
+}
+
 int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale,
                  int act_bits, int use_hadamard, uint16_t* Y, void* ws, size_t ws_bytes, cudaStream_t s,
                  DeviceState* d, bool ln = false, const float* gain = nullptr) {
@@ -590,6 +680,10 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   float* scales = reinterpret_cast<float*>(base + L.scales);
   int32_t* csum = reinterpret_cast<int32_t*>(base + L.csum);
   int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
+  if ((g_gemm_path == 0 || g_gemm_path == 6) && fused_fits(M, K, N)) {
+    const int fs = run_fused_decode(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, ln, gain, Y, d->sm_count, s);
+    if (fs != kFusedNotApplicable) return fs;
+  }
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
   if (st) return st;
   if (use_tc_path(M))
@@ -858,7 +952,7 @@ int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_t
 }
 
 int hbl_set_gemm_path(int path) {
-  if (path < 0 || path > 5) return HBL_ERR_INVALID_ARG;
+  if (path < 0 || path > 6) return HBL_ERR_INVALID_ARG;
   g_gemm_path = path;
   return HBL_OK;
 }

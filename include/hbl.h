@@ -255,18 +255,24 @@ int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_t
 int hbl_get_device_error(hbl_stream stream);
 
 /*
- * hbl_set_gemm_path -- which integer-GEMM kernel the forward and
- * hbl_gemm_codes use: 0 = by size (default: for M >= 128 tokens the tcgen05
- * tensor-core kernel with one 128 x 256 tile per CTA; for 9..64 tokens the
- * decode kernel split over K across a thread-block cluster (K >= 512); for
- * 1..8 tokens the decode kernel with one CTA per 16 rows; the warp-level
- * split-K kernel otherwise), 1 = always the warp-level split-K kernel,
- * 2 = always the persistent tcgen05 kernel (128 x 128 tiles), 3 = as 0 but
- * never the cluster or streaming decode kernels, 4 = always the one-tile
- * tcgen05 kernel, 5 = as 0 (the weight-streaming decode kernel is the default
- * for 1..16 tokens with K % 2048 == 0).
- * All give identical results; the knob exists to check and time each one.
- * Process-wide.
+ * hbl_set_gemm_path -- which kernels the forward and hbl_gemm_codes use:
+ * 0 = by size (default). The forward of 1..16 tokens with K in {2048, 4096}
+ * (or K = 8192 with at most 8 tokens) and N % 16 == 0 runs as ONE fused kernel
+ * (transform, quantiser, GEMM and dequant; codes exchanged between the CTAs
+ * of a thread-block cluster). Otherwise the quantiser kernel runs first and
+ * the GEMM is chosen by M: for M >= 128 tokens the tcgen05 tensor-core kernel
+ * with one 128 x 256 tile per CTA; for 1..16 tokens with K % 2048 == 0 the
+ * weight-streaming kernel (one CTA per SM); for 9..64 tokens the decode kernel
+ * split over K across a thread-block cluster (K >= 512); for 1..8 tokens the
+ * decode kernel with one CTA per 16 rows; the warp-level split-K kernel
+ * otherwise.
+ * 1 = always the warp-level split-K kernel, 2 = always the persistent tcgen05
+ * kernel (128 x 128 tiles), 3 = as 0 but never the fused, cluster or
+ * streaming decode kernels, 4 = always the one-tile tcgen05 kernel,
+ * 5 = as 0 but never the fused forward, 6 = as 0.
+ * All give results within the parity bounds of the oracle (the fused forward
+ * sums the transform in another order, so a code at a rounding tie may
+ * differ); the knob exists to check and time each one. Process-wide.
  */
 int hbl_set_gemm_path(int path);
 

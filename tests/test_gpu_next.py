@@ -63,6 +63,31 @@ def test_forward_ln(H, M, K, N, a, h):
     parity.check_y(Y.float().cpu().numpy(), ref["Y"], ref["s"], alpha, diff.sum(1))
 
 
+@pytest.mark.parametrize("M,K,N,a,h", [(16, 4096, 4096, 4, 1), (5, 4096, 512, 8, 0), (2, 8192, 64, 4, 1),
+                                       (11, 2048, 4096, 8, 1)])
+def test_forward_ln_fused_matches_two_kernel(H, M, K, N, a, h):
+    """With the RMSNorm prologue, the single-kernel decode forward gives the same
+    bits as the quantiser kernel + decode GEMM."""
+    from hadamard_bit_quant_b200 import layer
+    X = inputs.gaussian_with_outliers(M, K, 8, inputs.outlier_channels(K, 0.01, 4).tolist(), 50.0)
+    W = inputs.gaussian_weights(N, K, 9)
+    g = _gain(K, 3)
+    Wpk, wsc = layer.pack_weights(W.cuda())
+    ws = layer.workspace(M, K, N, "cuda")
+    out = {}
+    try:
+        for path in (6, 5):
+            H.hbl_set_gemm_path(path)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            H.hbl_forward_ln_ws(X.cuda(), M, K, N, g.cuda(), Wpk, wsc, a, h, Y, ws, ws.numel())
+            out[path] = Y
+    finally:
+        H.hbl_set_gemm_path(0)
+    torch.cuda.synchronize()
+    assert H.hbl_get_device_error() == 0
+    assert torch.equal(out[6], out[5])
+
+
 # ----------------------------------------------------------------------------- f2: rotated weights
 @pytest.mark.parametrize("N,K", [(64, 256), (256, 4096), (16, 16384)])
 def test_pack_weights_rotated(H, N, K):

@@ -268,6 +268,40 @@ def test_forward_paths(L, gemm_path, path):
     _forward_case(L, inputs.student_t(129, 1024, 1), inputs.gaussian_weights(80, 1024, 2), 8, 0)
 
 
+# ----------------------------------------------------------------------------- fused decode forward
+FUSED_SHAPES = [(1, 2048, 16, 4, 1), (2, 4096, 4096, 8, 1), (3, 4096, 48, 4, 0), (5, 8192, 2416, 4, 1),
+                (8, 8192, 256, 8, 0), (9, 2048, 4096, 4, 1), (16, 4096, 4096, 4, 1), (16, 4096, 4096, 8, 0),
+                (12, 2048, 16 * 1184, 8, 1), (16, 4096, 16 * 1200, 4, 1), (7, 4096, 1024, 4, 1)]
+
+
+@pytest.mark.parametrize("M,K,N,a,h", FUSED_SHAPES)
+def test_fused_forward_matches_two_kernel_path(L, gemm_path, M, K, N, a, h):
+    """The single-kernel decode forward (transform, quantiser, GEMM and dequant
+    with the codes exchanged inside a cluster) gives the same bits as the
+    quantiser kernel followed by each decode GEMM kernel; those are checked
+    against the oracle by the other forward and GEMM tests."""
+    from hadamard_bit_quant_b200 import hbl
+    X = inputs.gaussian_with_outliers(M, K, M + K, inputs.outlier_channels(K, 0.01, 1).tolist(), 50.0)
+    W = inputs.gaussian_weights(N, K, N + 1)
+    Wpk, wsc = L.pack_weights(dev(W))
+    Xd = dev(X)
+    out = {}
+    for path in (6, 5, 3):
+        gemm_path(path)
+        out[path] = L.forward(Xd, Wpk, wsc, N, a, h).clone()
+    torch.cuda.synchronize()
+    assert hbl.hbl_get_device_error() == 0
+    assert torch.equal(out[6], out[5])
+    assert torch.equal(out[6], out[3])
+
+
+@pytest.mark.parametrize("path", [5, 3], ids=["stream", "decode_no_cluster"])
+@pytest.mark.parametrize("case", inputs.decode_oproj_cases(), ids=lambda c: c.label)
+def test_forward_decode_two_kernel_paths(L, gemm_path, path, case):
+    gemm_path(path)
+    _forward_case(L, case.make_x(), case.make_w(), case.act_bits, case.use_hadamard)
+
+
 def test_chained_forwards_match_synchronised(L):
     """Back-to-back forwards on one stream, each consuming the previous output
     (programmatic dependent launches overlap their prologues), must give the
