@@ -42,7 +42,6 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = HBL_STREAM_STAGES;
 constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB: 4 boxes of [16][128 B]
 constexpr int kMaxGroups = 8;                      // per CTA
-constexpr int kBatch = 4;                          // groups whose MMAs are interleaved
 constexpr long long kSpinLimit = 4000000000ll;
 
 HBL_DEVINL uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -91,6 +90,98 @@ struct Layout {
   static constexpr size_t kRing = (size_t)kStages * kUnitBytes;
   static constexpr size_t kBytes = 1024 + kRing + 2 * (size_t)kCodeBuf + 256;
 };
+
+// Consumer side for a CTA that owns exactly NG groups: per chunk, wait for
+// the chunk's codes and all NG weight units, load every fragment, release the
+// slots, then issue the chunk's MMAs q by q over all groups (2*NG independent
+// accumulator chains; with one token tile, even and odd q accumulate
+// separately). Ends by writing this warp's partial sums into shared memory
+// (aliasing the ring) once every consumer warp is past its last unit.
+template <int NG, int TN, int MT>
+HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, uint64_t* wempty,
+                        uint64_t* cfull, uint64_t* cempty, volatile int* abort, int warp, int lane) {
+  using Lay = Layout<MT>;
+  constexpr int SPLIT = TN == 1 ? 2 : 1;
+  const int g = lane >> 2, tig = lane & 3;
+  const int ch = ((warp & 1) << 2) + tig;
+  int acc[NG][TN * SPLIT][4];
+#pragma unroll
+  for (int a = 0; a < NG; ++a)
+#pragma unroll
+    for (int i = 0; i < TN * SPLIT; ++i)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
+  bool ok = true;
+  for (int c = 0; c < nchunks && ok; ++c) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&cfull[c & 1], (uint32_t)(c >> 1) & 1u, abort))) { ok = false; break; }
+    const uint8_t* cb = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
+    uint2 bf[TN][8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int box = 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
+#pragma unroll
+      for (int i = 0; i < TN; ++i) {
+        const int m = 8 * i + g;
+        bf[i][q] = *reinterpret_cast<const uint2*>(cb + box * Lay::kCodeBox + m * 128 + ((cch ^ (m & 7)) << 4) +
+                                                   ((tig & 1) << 3));
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
+    uint32_t A4[NG][4], B4[NG][4];
+#pragma unroll
+    for (int b = 0; b < NG; ++b) {
+      const int u = c * NG + b;
+      const int s = u % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
+      const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
+      const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
+      const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+      A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
+      B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
+    }
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < NG; ++b) mbar_arrive(&wempty[(c * NG + b) % kStages]);
+    }
+    if (!ok) break;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int w = q >> 1, jj = 2 * (q & 1);
+#pragma unroll
+      for (int b = 0; b < NG; ++b) {
+        const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj), unpack_u8x4(A4[b][w], jj + 1),
+                               unpack_u8x4(B4[b][w], jj + 1)};
+#pragma unroll
+        for (int i = 0; i < TN; ++i) mma_u8s8_16832(acc[b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
+      }
+    }
+  }
+  if constexpr (SPLIT == 2) {
+#pragma unroll
+    for (int a = 0; a < NG; ++a)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
+  }
+  // partial sums of the 8 warps -> shared memory (aliases the ring, so only
+  // after every warp is done with it): red[warp][group][row][token]
+  asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers * 32) : "memory");
+  if (ok && *abort == 0) {
+    int* red = reinterpret_cast<int*>(ring);
+#pragma unroll
+    for (int gl = 0; gl < NG; ++gl)
+#pragma unroll
+      for (int i = 0; i < TN; ++i)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int row = g + ((r >> 1) << 3);
+          const int tok = 8 * i + 2 * tig + (r & 1);
+          red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
+        }
+  }
+  return ok;
+}
 
 template <int TN, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -189,104 +280,19 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   } else {
     // ----- consumers: warp w takes 256-k block w of every unit -----
-    // The MMAs of up to kBatch groups are interleaved q by q so that
-    // 2 * kBatch independent accumulator chains are in flight (with one token
-    // tile, even and odd q accumulate separately and are added at the end).
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-    const int g = lane >> 2, tig = lane & 3;
-    constexpr int SPLIT = TN == 1 ? 2 : 1;
-    int acc[kMaxGroups][TN * SPLIT][4];
-#pragma unroll
-    for (int a = 0; a < kMaxGroups; ++a)
-#pragma unroll
-      for (int i = 0; i < TN * SPLIT; ++i)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
     bool ok = true;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&cfull[c & 1], (uint32_t)(c >> 1) & 1u, abort))) { ok = false; break; }
-      const uint8_t* cb = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
-      // B fragments of this warp's block for this chunk (reused by every group)
-      uint2 bf[TN][8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int box = 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
-#pragma unroll
-        for (int i = 0; i < TN; ++i) {
-          const int m = 8 * i + g;
-          bf[i][q] = *reinterpret_cast<const uint2*>(cb + box * Lay::kCodeBox + m * 128 + ((cch ^ (m & 7)) << 4) +
-                                                     ((tig & 1) << 3));
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
-      const int ch = ((warp & 1) << 2) + tig;
-#pragma unroll
-      for (int gb = 0; gb < kMaxGroups; gb += kBatch) {
-        if (gb < ng && ok) {
-          uint32_t A4[kBatch][4], B4[kBatch][4];
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) {
-            if (gb + b < ng) {
-              const int u = c * ng + gb + b;
-              const int s = u % kStages;
-              if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
-              const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
-              const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
-              const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
-              A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
-              B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
-            }
-          }
-          __syncwarp();
-          if (lane == 0) {
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b)
-              if (gb + b < ng) mbar_arrive(&wempty[(c * ng + gb + b) % kStages]);
-          }
-          if (!ok) break;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int w = q >> 1, jj = 2 * (q & 1);
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-              if (gb + b < ng) {
-                const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj),
-                                       unpack_u8x4(A4[b][w], jj + 1), unpack_u8x4(B4[b][w], jj + 1)};
-#pragma unroll
-                for (int i = 0; i < TN; ++i)
-                  mma_u8s8_16832(acc[gb + b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
-              }
-            }
-          }
-        }
-      }
+    switch (ng) {
+      case 1: ok = consume<1, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      case 2: ok = consume<2, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      case 3: ok = consume<3, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      case 4: ok = consume<4, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      case 5: ok = consume<5, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      case 6: ok = consume<6, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      case 7: ok = consume<7, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
+      default: ok = consume<8, TN, MT>(nchunks, ring, cbuf, wfull, wempty, cfull, cempty, abort, warp, lane); break;
     }
-    if constexpr (SPLIT == 2) {
-#pragma unroll
-      for (int a = 0; a < kMaxGroups; ++a)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
-    }
-    // partial sums of the 8 warps -> shared memory (aliases the ring, so only
-    // after every warp is done with it): red[warp][group][row][token]
-    asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers * 32) : "memory");
-    if (ok && *abort == 0) {
-      int* red = reinterpret_cast<int*>(ring);
-#pragma unroll
-      for (int gl = 0; gl < kMaxGroups; ++gl) {
-        if (gl < ng) {
-#pragma unroll
-          for (int i = 0; i < TN; ++i)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int row = g + ((r >> 1) << 3);
-              const int tok = 8 * i + 2 * tig + (r & 1);
-              red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
-            }
-        }
-      }
-    }
+    (void)ok;
   }
   // every copy was consumed (or the CTA gave up); the ring may be reused
   const bool all_ok = __syncthreads_and(*abort == 0) != 0;

@@ -395,11 +395,6 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 // takes the fused single-kernel decode wherever it fits; 0 does the same)
 int g_gemm_path = 0;
 
-bool use_tc_path(int M) {
-  if (g_gemm_path == 1) return false;
-  if (g_gemm_path == 2 || g_gemm_path == 4) return true;
-  return M >= 128;
-}
 
 // Persistent tcgen05 kernel (one CTA per SM, 128 x 128 tiles, double-buffered accumulator).
 int run_gemm_tc2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
@@ -444,6 +439,34 @@ int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, co
 
 bool decode_path_fits(int M, int K) {
   return M <= kLatencyTokens && dec::smem_bytes(K, 8) <= 200 * 1024;
+}
+
+enum class GemmKind { Decode, Mma, Tc, Tc2 };
+
+// Which GEMM kernel runs (after the quantiser). By size, from timings on B200
+// over M in 1..4096 and K, N in 2048..16384:
+//  * 1..16 tokens stream the weights (decode kernels);
+//  * up to 32 tokens, and with N < 8192 up to 255 tokens (N <= 2048: up to
+//    1023), the split-K warp-level kernel: it keeps every SM busy where the
+//    tensor-core kernels would have few 128-row tiles;
+//  * K >= 8192 with at least 256 tiles of 128 x 128: the tcgen05 kernel with
+//    one 128 x 256 tile per CTA (half the weight re-reads of 128-token tiles);
+//  * otherwise the persistent tcgen05 kernel (128 x 128 tiles, accumulator
+//    double-buffered so the epilogue overlaps the next tile).
+GemmKind choose_gemm(int M, int K, int N) {
+  switch (g_gemm_path) {
+    case 1: return GemmKind::Mma;
+    case 2: return GemmKind::Tc2;
+    case 4: return GemmKind::Tc;
+    default: break;
+  }
+  if (M <= 16 && decode_path_fits(M, K)) return GemmKind::Decode;
+  if (M <= 32) return GemmKind::Mma;
+  const long long tiles = (long long)((N + 127) / 128) * ((M + 127) / 128);
+  if (K >= 8192 && tiles >= 256) return GemmKind::Tc;
+  if (N >= 8192) return GemmKind::Tc2;
+  if (M < 256 || (N <= 2048 && M < 1024)) return GemmKind::Mma;
+  return GemmKind::Tc2;
 }
 
 #ifndef HBL_DECODE_MAX_CLUSTER
@@ -593,7 +616,17 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 // ---------------------------------------------------------------------------
 constexpr int kFusedNotApplicable = -1;
 
-int fused_cluster_size(int M) { return M <= 2 ? 1 : (M <= 4 ? 2 : (M <= 8 ? 4 : 8)); }
+#ifndef HBL_FUSED_CS_MAX
+#define HBL_FUSED_CS_MAX 8
+#endif
+#ifndef HBL_FUSED_BALANCE
+#define HBL_FUSED_BALANCE 0
+#endif
+int fused_cluster_size(int M) {
+  int cs = M <= 2 ? 1 : (M <= 4 ? 2 : (M <= 8 ? 4 : 8));
+  if (HBL_FUSED_CS_MAX >= 16 && M > 8) cs = 16;
+  return cs < HBL_FUSED_CS_MAX ? cs : HBL_FUSED_CS_MAX;
+}
 
 template <int LOG_K, int TN>
 int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const float* gain, const float* alpha,
@@ -601,6 +634,13 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   auto* kern = fdec::fused_decode_kernel<LOG_K, TN>;
   const size_t smem = fdec::Layout<LOG_K, 8 * TN>::kBytes;
   ensure_smem_attr(kern, smem);
+  if (HBL_FUSED_CS_MAX > 8) {
+    static bool once = false;
+    if (!once) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      once = true;
+    }
+  }
   const int CS = fused_cluster_size(M);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
@@ -639,6 +679,12 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   if (grid > sm_count / CS * CS) grid = sm_count / CS * CS;
   const int groups = N / fdec::kGroupRows;
   if (grid < CS || groups > fdec::kMaxGroups * grid) return kFusedNotApplicable;
+  if (HBL_FUSED_BALANCE) {
+    // every CTA the same number of 16-row groups: the next layer waits for the slowest
+    const int ng = (groups + grid - 1) / grid;
+    const int need = (groups + ng - 1) / ng;
+    grid = (need + CS - 1) / CS * CS;
+  }
   cfg.gridDim = dim3((unsigned)grid);
   ProfScope ps("fused_decode", s);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, X, M, N, gain, alpha, flags, Y);
@@ -686,11 +732,12 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   }
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
   if (st) return st;
-  if (use_tc_path(M))
-    return g_gemm_path == 2 ? run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s)
-                            : run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
-  if (g_gemm_path != 1 && decode_path_fits(M, K))
-    return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count);
+  switch (choose_gemm(M, K, N)) {
+    case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
+    case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
+    case GemmKind::Decode: return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count);
+    case GemmKind::Mma: break;
+  }
   st = run_gemm(codes, M, K, N, Wpk, D, d->sm_count, s);
   if (st) return st;
   const long long total8 = (long long)M * N / 8;
@@ -867,11 +914,12 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   }
   code_rowsum_kernel<<<M, 256, 0, s>>>(codes, K, csum);
   if ((st = launch_status())) return st;
-  if (use_tc_path(M))
-    return g_gemm_path == 2 ? run_gemm_tc2(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s)
-                            : run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
-  if (g_gemm_path != 1 && decode_path_fits(M, K))
-    return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count);
+  switch (choose_gemm(M, K, N)) {
+    case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
+    case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
+    case GemmKind::Decode: return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count);
+    case GemmKind::Mma: break;
+  }
   if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
   sub_rowsum_kernel<<<(unsigned)(((long long)M * N + 255) / 256), 256, 0, s>>>(acc, csum, M, N);
   return launch_status();

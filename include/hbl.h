@@ -260,19 +260,20 @@ int hbl_get_device_error(hbl_stream stream);
  * (or K = 8192 with at most 8 tokens) and N % 16 == 0 runs as ONE fused kernel
  * (transform, quantiser, GEMM and dequant; codes exchanged between the CTAs
  * of a thread-block cluster). Otherwise the quantiser kernel runs first and
- * the GEMM is chosen by M: for M >= 128 tokens the tcgen05 tensor-core kernel
- * with one 128 x 256 tile per CTA; for 1..16 tokens with K % 2048 == 0 the
- * weight-streaming kernel (one CTA per SM); for 9..64 tokens the decode kernel
- * split over K across a thread-block cluster (K >= 512); for 1..8 tokens the
- * decode kernel with one CTA per 16 rows; the warp-level split-K kernel
- * otherwise.
+ * the GEMM is chosen by size: 1..16 tokens stream the weights (the
+ * weight-streaming kernel when K % 2048 == 0, else the decode kernel split
+ * over K across a cluster for 9..16 tokens, or with one CTA per 16 rows);
+ * up to 32 tokens, and with N < 8192 up to 255 tokens (N <= 2048: up to
+ * 1023), the warp-level split-K kernel; with K >= 8192 and at least 256
+ * tiles of 128 x 128, the tcgen05 kernel with one 128 x 256 tile per CTA;
+ * otherwise the persistent tcgen05 kernel (128 x 128 tiles).
  * 1 = always the warp-level split-K kernel, 2 = always the persistent tcgen05
- * kernel (128 x 128 tiles), 3 = as 0 but never the fused, cluster or
- * streaming decode kernels, 4 = always the one-tile tcgen05 kernel,
- * 5 = as 0 but never the fused forward, 6 = as 0.
+ * kernel, 3 = as 0 but never the fused, cluster or streaming decode kernels,
+ * 4 = always the one-tile tcgen05 kernel, 5 = as 0 but never the fused
+ * forward, 6 = as 0.
  * All give results within the parity bounds of the oracle (the fused forward
- * sums the transform in another order, so a code at a rounding tie may
- * differ); the knob exists to check and time each one. Process-wide.
+ * and the quantiser kernel share their summation order, so the paths give the
+ * same bits); the knob exists to check and time each one. Process-wide.
  */
 int hbl_set_gemm_path(int path);
 
