@@ -14,18 +14,24 @@
 //     a TMA ring from the first instruction on, before the kernel waits for
 //     the grid that produced X (programmatic dependent launch);
 //   * the 8 consumer warps of cluster rank r transform and quantise token rows
-//     r, r + CS, ... (two rows at a time, 256 threads per row, E = K/256
-//     values per thread, butterflies in registers, passes exchanged through
-//     padded shared memory), then write each row's codes, its scale and its
-//     per-warp code sums into the shared memory of EVERY CTA of the cluster
-//     (distributed shared memory). After a cluster barrier each CTA holds all
-//     M x K codes;
+//     2r and 2r + 1 (256 threads per row, E = K/256 values per thread,
+//     butterflies in registers, passes exchanged through padded shared
+//     memory) into this CTA's shared memory: codes row-contiguous, scale and
+//     per-warp code sums beside them. Lane 0 of warp q then sends both rows to
+//     cluster rank q (every rank but this one) with two bulk copies (shared memory to
+//     distributed shared memory, completing as transaction bytes on the
+//     peer's mbarrier). Each CTA waits on its own barrier for the M - 2 rows
+//     it receives, so it holds all M x K codes;
 //   * the consumers then run the m16n8k32 MMAs of their groups (weights as A,
 //     u = t + 1 unpacked in registers; codes as B), batches of groups
 //     interleaved for independent accumulator chains, add the 8 warps' partial
 //     sums in shared memory, subtract the code sums and store bf16.
-// Every mbarrier wait is bounded; a CTA that gives up sets the device error
-// word, still takes part in both cluster barriers, and writes no output.
+// Two cluster barriers: #1 (arrive at start, wait before the first copy) makes
+// sure every peer runs and has armed its barrier; #2 (arrive once this CTA's
+// rows have all landed, wait at exit) keeps every CTA's shared memory alive
+// until the copies out of it have completed. Every mbarrier wait is bounded;
+// a CTA that gives up sets the device error word, still takes part in both
+// cluster barriers, and writes no output.
 #pragma once
 #include <cuda.h>
 #include "hbl_common.cuh"
@@ -43,9 +49,9 @@ constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = 8;
 constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB = 4 boxes of [16][128 B]
 constexpr int kMaxGroups = 8;
-constexpr int kBatch = 4;
 constexpr int kRowBatch = 2;                        // token rows transformed together
 constexpr int kMaxTokens = 16;
+constexpr int kMetaBytes = 48;                      // scale + 8 per-warp code sums, padded to 16 B
 constexpr long long kSpinLimit = 4000000000ll;
 
 __host__ __device__ constexpr int ilog2_c(int x) { return x <= 1 ? 0 : 1 + ilog2_c(x / 2); }
@@ -103,16 +109,15 @@ HBL_DEVINL uint32_t map_rank(uint32_t local_addr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(local_addr), "r"(rank));
   return r;
 }
-HBL_DEVINL void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to a
+// peer's (addresses from mapa), completing as transaction bytes on the
+// peer's mbarrier.
+HBL_DEVINL void bulk_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t peer_bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+               "r"(su32(src)), "r"(bytes), "r"(peer_bar)
                : "memory");
 }
-HBL_DEVINL void st_cluster_v2(uint32_t addr, uint32_t a, uint32_t b) {
-  asm volatile("st.shared::cluster.v2.u32 [%0], {%1, %2};\n" ::"r"(addr), "r"(a), "r"(b) : "memory");
-}
-HBL_DEVINL void st_cluster_u32(uint32_t addr, uint32_t a) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(addr), "r"(a) : "memory");
-}
+HBL_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 HBL_DEVINL void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory"); }
 HBL_DEVINL void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
 HBL_DEVINL void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
@@ -129,20 +134,21 @@ struct Layout {
   static constexpr size_t kX = (size_t)kRowBatch * KPAD * 4;
   static constexpr size_t oCodes = kRing;
   static constexpr size_t oX = oCodes + kCodes;
-  static constexpr size_t oScale = oX + kX;                   // float [kMaxTokens]
-  static constexpr size_t oCsum = oScale + kMaxTokens * 4;    // int [kMaxTokens][kConsumers]
-  static constexpr size_t oRed = oCsum + kMaxTokens * kConsumers * 4;   // float [kRowBatch * 2][kConsumers]
+  static constexpr size_t oMeta = oX + kX;                    // per token: scale, 8 code sums, pad (48 B)
+  static constexpr size_t oRed = oMeta + kMaxTokens * kMetaBytes;   // float [kRowBatch * 2][kConsumers]
   static constexpr size_t oBars = oRed + kRowBatch * 2 * kConsumers * 4;
-  static constexpr size_t kBytes = 1024 + oBars + 2 * kStages * 8 + 16;
+  static constexpr size_t kBytes = 1024 + oBars + (2 * kStages + 1) * 8 + 16;
   static_assert(kMaxGroups * kConsumers * kGroupRows * MT * 4 <= kRing, "reduction must fit in the ring");
 };
 
 // Byte offset of the 16-byte code chunk holding k = 16*c16 .. 16*c16+15 of
-// token m: box k/128 of [MT][128 B], 128B-swizzled by m % 8 (the layout a
-// TMA SWIZZLE_128B load of a [MT][128] box produces).
-template <int MT>
+// token m: token rows are contiguous (K bytes each, so a row moves between
+// CTAs as one bulk copy); within each 128-byte segment the eight 16-byte
+// chunks are permuted by XOR with m % 8, which keeps the MMA fragment reads
+// (8 tokens x one chunk) free of bank conflicts.
+template <int K>
 HBL_DEVINL uint32_t code_off(int m, int c16) {
-  return (uint32_t)((c16 >> 3) * (MT * 128) + m * 128 + (((c16 & 7) ^ (m & 7)) << 4));
+  return (uint32_t)(m * K + (c16 >> 3) * 128 + (((c16 & 7) ^ (m & 7)) << 4));
 }
 
 // Sum (or max) over the 256 consumer threads of NR values at once (one
@@ -171,15 +177,12 @@ HBL_DEVINL void rows_reduce_n(float (&x)[NR], float* slot) {
   }
 }
 
-// Phase 1 for NR (1 or 2) token rows m0, m0 + cs: load, optional RMSNorm,
-// optional transform, quantise, and write codes, scale and per-warp code sums
-// into the shared memory of every CTA of the cluster (of this CTA alone when
-// cs == 1). `cw1` is true until this CTA has waited on cluster barrier #1,
-// which must precede the first remote store.
+// Phase 1 for NR (1 or 2) token rows m0, m0 + 1: load, optional RMSNorm,
+// optional transform, quantise, and write the codes, the scale and the
+// per-warp code sums of each row into this CTA's shared memory.
 template <int LOG_K, int MT, int NR>
-HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, uint32_t cs, bool had, bool int8, bool ln,
-                           const float* __restrict__ gain, float* xb, float* s_red, uint8_t* cbuf, float* s_scale,
-                           int* s_csum, bool& cw1) {
+HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, bool had, bool int8, bool ln,
+                           const float* __restrict__ gain, float* xb, float* s_red, uint8_t* cbuf, uint32_t* meta) {
   constexpr int K = 1 << LOG_K, E = K / kRowThreads, G = ilog2_c(E), P = (LOG_K + G - 1) / G, KPAD = K + K / E;
   constexpr int T = kRowThreads;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -189,7 +192,7 @@ HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, uint32_t cs, 
   // load of a row is in flight at once
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
-    const uint16_t* xr = X + (size_t)(m0 + r * (int)cs) * K;
+    const uint16_t* xr = X + (size_t)(m0 + r) * K;
     nrm[r] = 1.f;
     if (had) {
 #pragma unroll
@@ -286,13 +289,9 @@ HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, uint32_t cs, 
   consumers_sync();   // the slots' previous readers are done
   if (int8) rows_reduce_n<NR, true>(stat, s_red + 2 * kConsumers);
   else rows_reduce_n<NR, false>(stat, s_red + 2 * kConsumers);
-  if (cw1) {
-    cluster_wait();   // #1: every peer runs, so its shared memory may be written
-    cw1 = false;
-  }
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
-    const int m = m0 + r * (int)cs;
+    const int m = m0 + r;
     const float rs = __fmul_rn(stat[r], nrm[r]);
     float mult, scale;
     int lo, hi;
@@ -322,36 +321,105 @@ HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, uint32_t cs, 
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) csum += __shfl_xor_sync(0xffffffffu, csum, off);
-    if (cs == 1) {
-      if constexpr (E == 8) {
-        *reinterpret_cast<uint2*>(cbuf + code_off<MT>(m, t >> 1) + ((t & 1) << 3)) = make_uint2(packed[0], packed[1]);
-      } else {
-#pragma unroll
-        for (int h = 0; h < E / 16; ++h)
-          *reinterpret_cast<uint4*>(cbuf + code_off<MT>(m, t * (E / 16) + h)) =
-              make_uint4(packed[4 * h], packed[4 * h + 1], packed[4 * h + 2], packed[4 * h + 3]);
-      }
-      if (lane == 0) s_csum[m * kConsumers + warp] = csum;
-      if (t == 0) s_scale[m] = scale;
+    if constexpr (E == 8) {
+      *reinterpret_cast<uint2*>(cbuf + code_off<K>(m, t >> 1) + ((t & 1) << 3)) = make_uint2(packed[0], packed[1]);
     } else {
-      const uint32_t scale_bits = __float_as_uint(scale);
-      for (uint32_t q = 0; q < cs; ++q) {
-        if constexpr (E == 8) {
-          const uint32_t off = code_off<MT>(m, t >> 1) + ((t & 1) << 3);
-          st_cluster_v2(map_rank(su32(cbuf + off), q), packed[0], packed[1]);
-        } else {
 #pragma unroll
-          for (int h = 0; h < E / 16; ++h) {
-            const uint32_t off = code_off<MT>(m, t * (E / 16) + h);
-            st_cluster_v4(map_rank(su32(cbuf + off), q), packed[4 * h], packed[4 * h + 1], packed[4 * h + 2],
-                          packed[4 * h + 3]);
-          }
-        }
-        if (lane == 0) st_cluster_u32(map_rank(su32(s_csum + m * kConsumers + warp), q), (uint32_t)csum);
-        if (t == 0) st_cluster_u32(map_rank(su32(s_scale + m), q), scale_bits);
+      for (int h = 0; h < E / 16; ++h)
+        *reinterpret_cast<uint4*>(cbuf + code_off<K>(m, t * (E / 16) + h)) =
+            make_uint4(packed[4 * h], packed[4 * h + 1], packed[4 * h + 2], packed[4 * h + 3]);
+    }
+    uint32_t* mrow = meta + m * (kMetaBytes / 4);
+    if (lane == 0) mrow[1 + warp] = (uint32_t)csum;
+    if (t == 0) mrow[0] = __float_as_uint(scale);
+  }
+}
+
+// Phase 2 for a CTA that owns exactly NG groups: per 2048-k chunk, wait for
+// all NG weight units, load every fragment, release the slots, then issue the
+// chunk's MMAs q by q over all groups (2*NG independent accumulator chains;
+// with one token tile, even and odd q accumulate separately). Codes are read
+// from the resident row-major buffer. Ends by writing this warp's partial sums
+// into shared memory (aliasing the ring) once every consumer is past its last
+// unit: red[warp][group][row][token].
+template <int NG, int TN, int K>
+HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, uint64_t* wempty, volatile int* abort,
+                          int warp, int lane) {
+  constexpr int MT = 8 * TN;
+  constexpr int nchunks = K / kChunk;
+  constexpr int SPLIT = TN == 1 ? 2 : 1;
+  const int g = lane >> 2, tig = lane & 3;
+  const int ch = ((warp & 1) << 2) + tig;
+  int acc[NG][TN * SPLIT][4];
+#pragma unroll
+  for (int a = 0; a < NG; ++a)
+#pragma unroll
+    for (int i = 0; i < TN * SPLIT; ++i)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
+  bool ok = true;
+  for (int c = 0; c < nchunks && ok; ++c) {
+    uint2 bf[TN][8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int box = c * (kChunk / 128) + 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
+#pragma unroll
+      for (int i = 0; i < TN; ++i) {
+        const int m = 8 * i + g;
+        bf[i][q] = *reinterpret_cast<const uint2*>(cbuf + m * K + box * 128 + ((cch ^ (m & 7)) << 4) + ((tig & 1) << 3));
+      }
+    }
+    uint32_t A4[NG][4], B4[NG][4];
+#pragma unroll
+    for (int b = 0; b < NG; ++b) {
+      const int u = c * NG + b;
+      const int s = u % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
+      const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
+      const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
+      const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+      A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
+      B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
+    }
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < NG; ++b) mbar_arrive(&wempty[(c * NG + b) % kStages]);
+    }
+    if (!ok) break;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int w = q >> 1, jj = 2 * (q & 1);
+#pragma unroll
+      for (int b = 0; b < NG; ++b) {
+        const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj), unpack_u8x4(A4[b][w], jj + 1),
+                               unpack_u8x4(B4[b][w], jj + 1)};
+#pragma unroll
+        for (int i = 0; i < TN; ++i) mma_u8s8_16832(acc[b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
       }
     }
   }
+  if constexpr (SPLIT == 2) {
+#pragma unroll
+    for (int a = 0; a < NG; ++a)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
+  }
+  consumers_sync();   // every consumer is past its last unit: the ring may be reused
+  if (ok && *abort == 0) {
+    int* red = reinterpret_cast<int*>(ring);
+#pragma unroll
+    for (int gl = 0; gl < NG; ++gl)
+#pragma unroll
+      for (int i = 0; i < TN; ++i)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int row = g + ((r >> 1) << 3);
+          const int tok = 8 * i + 2 * tig + (r & 1);
+          red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
+        }
+  }
+  return ok;
 }
 
 // flags: bit 0 use_hadamard, bit 1 INT8 (else INT4), bit 2 RMSNorm prologue.
@@ -368,12 +436,12 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
   uint8_t* ring = base;
   uint8_t* cbuf = base + Lay::oCodes;
   float* xb = reinterpret_cast<float*>(base + Lay::oX);
-  float* s_scale = reinterpret_cast<float*>(base + Lay::oScale);
-  int* s_csum = reinterpret_cast<int*>(base + Lay::oCsum);
+  uint32_t* meta = reinterpret_cast<uint32_t*>(base + Lay::oMeta);
   float* s_red = reinterpret_cast<float*>(base + Lay::oRed);
   uint64_t* wfull = reinterpret_cast<uint64_t*>(base + Lay::oBars);
   uint64_t* wempty = wfull + kStages;
-  volatile int* abort = reinterpret_cast<volatile int*>(wempty + kStages);
+  uint64_t* codes_full = wempty + kStages;   // the peers' rows have landed
+  volatile int* abort = reinterpret_cast<volatile int*>(codes_full + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_rank(), csize = cluster_size();
@@ -381,18 +449,25 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
   const int Gd = gridDim.x;
   const int ng = (groups - (int)blockIdx.x + Gd - 1) / Gd;
   const int units = nchunks * ng;
+  // token rows [m0, m0 + nr) are transformed and quantised by this CTA
+  const int m0 = (int)crank * kRowBatch;
+  const int nr = M - m0 < 0 ? 0 : (M - m0 > kRowBatch ? kRowBatch : M - m0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], kConsumers);
     }
+    mbar_init(codes_full, 1);
+    // every other row arrives from a peer: codes (K bytes) + scale and code sums
+    if (csize > 1) mbar_expect_tx(codes_full, (uint32_t)((M - nr) * (Lay::K + kMetaBytes)));
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  if (csize > 1) cluster_arrive_relaxed();   // #1: this CTA runs (peers may write its shared memory after #1)
+  // #1: this CTA runs and its codes barrier is armed (peers may copy into it after #1)
+  if (csize > 1) cluster_arrive_relaxed();
 
   if (warp == kConsumers) {
     // ----- producer: the weight ring (independent of the previous grid) -----
@@ -411,7 +486,7 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
     __syncwarp();
     if (csize > 1) {
       cluster_wait();             // #1
-      cluster_arrive_relaxed();   // #2: the producer writes nothing a peer reads
+      cluster_arrive_relaxed();   // #2: the producer receives no rows
     }
     if (lane == 0) {
       bool ok = true;
@@ -434,110 +509,38 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
     const bool had = (flags & 1) != 0, int8 = (flags & 2) != 0, ln = (flags & 4) != 0;
     asm volatile("griddepcontrol.wait;\n" ::: "memory");   // X is ready past this point
     const float a_w = __ldg(alpha);
-    bool cw1 = csize > 1;
-    for (int m0 = (int)crank; m0 < M; m0 += (int)csize * kRowBatch) {
-      if (m0 + (int)csize < M)
-        rows_phase<LOG_K, MT, 2>(X, m0, csize, had, int8, ln, gain, xb, s_red, cbuf, s_scale, s_csum, cw1);
-      else
-        rows_phase<LOG_K, MT, 1>(X, m0, csize, had, int8, ln, gain, xb, s_red, cbuf, s_scale, s_csum, cw1);
-    }
+    if (nr == 2) rows_phase<LOG_K, MT, 2>(X, m0, had, int8, ln, gain, xb, s_red, cbuf, meta);
+    else if (nr == 1) rows_phase<LOG_K, MT, 1>(X, m0, had, int8, ln, gain, xb, s_red, cbuf, meta);
+    fence_proxy_async_smem();   // the rows written here are read next by the bulk-copy engine
+    consumers_sync();           // ... and by every consumer warp
+    bool ok = true;
     if (csize > 1) {
-      if (cw1) cluster_wait();   // #1 (this CTA had no rows)
-      cluster_arrive_release();  // #2: this CTA's writes into the cluster are done
-      cluster_wait();            // #2: every row of codes is here
-    } else {
-      consumers_sync();          // every row of codes is here
+      cluster_wait();   // #1: every peer runs and has armed its codes barrier
+      // lane 0 of warp w sends to peer w (warp 0 to peer csize - 1 ... all peers but this CTA)
+      const uint32_t q = (uint32_t)warp;
+      if (lane == 0 && nr > 0 && q < csize && q != crank) {
+        const uint32_t bar = map_rank(su32(codes_full), q);
+        const uint32_t cb_off = (uint32_t)m0 * Lay::K, mt_off = (uint32_t)m0 * kMetaBytes;
+        bulk_to_peer(map_rank(su32(cbuf + cb_off), q), cbuf + cb_off, (uint32_t)nr * Lay::K, bar);
+        bulk_to_peer(map_rank(su32(reinterpret_cast<uint8_t*>(meta) + mt_off), q),
+                     reinterpret_cast<uint8_t*>(meta) + mt_off, (uint32_t)nr * kMetaBytes, bar);
+      }
+      // the peers' rows
+      ok = __all_sync(0xffffffffu, mbar_wait(codes_full, 0u, abort)) != 0;
+      cluster_arrive_relaxed();   // #2: every row this CTA receives has landed
     }
 
     // ----- consumers, phase 2: MMAs over the weight ring -----
-    const int g = lane >> 2, tig = lane & 3;
-    constexpr int SPLIT = TN == 1 ? 2 : 1;
-    int acc[kMaxGroups][TN * SPLIT][4];
-#pragma unroll
-    for (int a = 0; a < kMaxGroups; ++a)
-#pragma unroll
-      for (int i = 0; i < TN * SPLIT; ++i)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) acc[a][i][r] = 0;
-    bool ok = true;
-    const int ch = ((warp & 1) << 2) + tig;
-    for (int c = 0; c < nchunks && ok; ++c) {
-      uint2 bf[TN][8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int box = c * (kChunk / 128) + 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
-#pragma unroll
-        for (int i = 0; i < TN; ++i) {
-          const int m = 8 * i + g;
-          bf[i][q] = *reinterpret_cast<const uint2*>(cbuf + box * (MT * 128) + m * 128 + ((cch ^ (m & 7)) << 4) +
-                                                     ((tig & 1) << 3));
-        }
-      }
-#pragma unroll
-      for (int gb = 0; gb < kMaxGroups; gb += kBatch) {
-        if (gb < ng && ok) {
-          uint32_t A4[kBatch][4], B4[kBatch][4];
-#pragma unroll
-          for (int b = 0; b < kBatch; ++b) {
-            if (gb + b < ng) {
-              const int u = c * ng + gb + b;
-              const int s = u % kStages;
-              if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
-              const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
-              const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
-              const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
-              A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
-              B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
-            }
-          }
-          __syncwarp();
-          if (lane == 0) {
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b)
-              if (gb + b < ng) mbar_arrive(&wempty[(c * ng + gb + b) % kStages]);
-          }
-          if (!ok) break;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int w = q >> 1, jj = 2 * (q & 1);
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-              if (gb + b < ng) {
-                const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj),
-                                       unpack_u8x4(A4[b][w], jj + 1), unpack_u8x4(B4[b][w], jj + 1)};
-#pragma unroll
-                for (int i = 0; i < TN; ++i)
-                  mma_u8s8_16832(acc[gb + b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
-              }
-            }
-          }
-        }
-      }
-    }
-    if constexpr (SPLIT == 2) {
-#pragma unroll
-      for (int a = 0; a < kMaxGroups; ++a)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
-    }
-    // partial sums of the 8 warps -> shared memory, aliasing the ring once
-    // every consumer is past its last unit: red[warp][group][row][token]
-    consumers_sync();
-    if (ok && *abort == 0) {
-      int* red = reinterpret_cast<int*>(ring);
-#pragma unroll
-      for (int gl = 0; gl < kMaxGroups; ++gl) {
-        if (gl < ng) {
-#pragma unroll
-          for (int i = 0; i < TN; ++i)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int row = g + ((r >> 1) << 3);
-              const int tok = 8 * i + 2 * tig + (r & 1);
-              red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
-            }
-        }
-      }
+    switch (ok ? ng : 0) {
+      case 1: ok = fused_mma<1, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 2: ok = fused_mma<2, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 3: ok = fused_mma<3, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 4: ok = fused_mma<4, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 5: ok = fused_mma<5, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 6: ok = fused_mma<6, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 7: ok = fused_mma<7, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      case 8: ok = fused_mma<8, TN, Lay::K>(ring, cbuf, wfull, wempty, abort, warp, lane); break;
+      default: consumers_sync(); break;   // no groups (or no codes): keep the barrier count
     }
     consumers_sync();
     if (ok && *abort == 0) {
@@ -551,15 +554,19 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
           int s = 0;
 #pragma unroll
           for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * kGroupRows + row) * MT + tok];
+          const uint32_t* mrow = meta + tok * (kMetaBytes / 4);
           int cs = 0;
 #pragma unroll
-          for (int w = 0; w < kConsumers; ++w) cs += s_csum[tok * kConsumers + w];
+          for (int w = 0; w < kConsumers; ++w) cs += (int)mrow[1 + w];
           s -= cs;
-          const float y = __fmul_rn(__fmul_rn((float)s, s_scale[tok]), a_w);
+          const float y = __fmul_rn(__fmul_rn((float)s, __uint_as_float(mrow[0])), a_w);
           Y[(size_t)tok * N + n] = float_to_bf16_bits(y);
         }
       }
     }
+    // #2: every copy into every CTA of the cluster has landed, so the rows this
+    // CTA sent have been read and its shared memory may be released
+    if (csize > 1) cluster_wait();
   }
 }
 

@@ -616,17 +616,8 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 // ---------------------------------------------------------------------------
 constexpr int kFusedNotApplicable = -1;
 
-#ifndef HBL_FUSED_CS_MAX
-#define HBL_FUSED_CS_MAX 8
-#endif
-#ifndef HBL_FUSED_BALANCE
-#define HBL_FUSED_BALANCE 0
-#endif
-int fused_cluster_size(int M) {
-  int cs = M <= 2 ? 1 : (M <= 4 ? 2 : (M <= 8 ? 4 : 8));
-  if (HBL_FUSED_CS_MAX >= 16 && M > 8) cs = 16;
-  return cs < HBL_FUSED_CS_MAX ? cs : HBL_FUSED_CS_MAX;
-}
+// Cluster size of the fused decode kernel: each CTA transforms two token rows.
+int fused_cluster_size(int M) { return M <= 2 ? 1 : (M <= 4 ? 2 : (M <= 8 ? 4 : 8)); }
 
 template <int LOG_K, int TN>
 int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const float* gain, const float* alpha,
@@ -634,13 +625,6 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   auto* kern = fdec::fused_decode_kernel<LOG_K, TN>;
   const size_t smem = fdec::Layout<LOG_K, 8 * TN>::kBytes;
   ensure_smem_attr(kern, smem);
-  if (HBL_FUSED_CS_MAX > 8) {
-    static bool once = false;
-    if (!once) {
-      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      once = true;
-    }
-  }
   const int CS = fused_cluster_size(M);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
@@ -678,13 +662,7 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   int grid = clusters * CS;
   if (grid > sm_count / CS * CS) grid = sm_count / CS * CS;
   const int groups = N / fdec::kGroupRows;
-  if (grid < CS || groups > fdec::kMaxGroups * grid) return kFusedNotApplicable;
-  if (HBL_FUSED_BALANCE) {
-    // every CTA the same number of 16-row groups: the next layer waits for the slowest
-    const int ng = (groups + grid - 1) / grid;
-    const int need = (groups + ng - 1) / ng;
-    grid = (need + CS - 1) / CS * CS;
-  }
+  if (grid < CS || groups > fdec::kMaxGroups * grid || CS * fdec::kRowBatch < M) return kFusedNotApplicable;
   cfg.gridDim = dim3((unsigned)grid);
   ProfScope ps("fused_decode", s);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, X, M, N, gain, alpha, flags, Y);
