@@ -182,37 +182,52 @@ HBL_DEVINL void rows_reduce_n(float (&x)[NR], float* slot) {
 // per-warp code sums of each row into this CTA's shared memory.
 template <int LOG_K, int MT, int NR>
 HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, bool had, bool int8, bool ln,
-                           const float* __restrict__ gain, float* xb, float* s_red, uint8_t* cbuf, uint32_t* meta) {
+                           const float* __restrict__ gain, float* xb, float* s_red, uint8_t* cbuf, uint32_t* meta,
+                           bool wait1) {
   constexpr int K = 1 << LOG_K, E = K / kRowThreads, G = ilog2_c(E), P = (LOG_K + G - 1) / G, KPAD = K + K / E;
   constexpr int T = kRowThreads;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   float v[NR][E];
   float nrm[NR];
   // loads: the flag branches stay outside the unrolled loops so that every
-  // load of a row is in flight at once
+  // load of a row is in flight at once; `wait1` runs the cluster barrier wait
+  // while they are
+  if (had) {
+    uint32_t raw[NR][E];
 #pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    const uint16_t* xr = X + (size_t)(m0 + r) * K;
-    nrm[r] = 1.f;
-    if (had) {
+    for (int r = 0; r < NR; ++r) {
+      const uint16_t* xr = X + (size_t)(m0 + r) * K;
 #pragma unroll
-      for (int j = 0; j < E; ++j) v[r][j] = bf16_bits_to_float(__ldg(xr + t + j * T));
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(xr + (size_t)E * t);
-      uint4 w4[E / 8];
+      for (int j = 0; j < E; ++j) raw[r][j] = __ldg(xr + t + j * T);
+    }
+    if (wait1) cluster_wait();
 #pragma unroll
-      for (int q = 0; q < E / 8; ++q) w4[q] = __ldg(src + q);
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+      for (int j = 0; j < E; ++j) v[r][j] = __uint_as_float(raw[r][j] << 16);
+  } else {
+    uint4 w4[NR][E / 8];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const uint4* src = reinterpret_cast<const uint4*>(X + (size_t)(m0 + r) * K + (size_t)E * t);
+#pragma unroll
+      for (int q = 0; q < E / 8; ++q) w4[r][q] = __ldg(src + q);
+    }
+    if (wait1) cluster_wait();
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
 #pragma unroll
       for (int q = 0; q < E / 8; ++q) {
-        const uint32_t w[4] = {w4[q].x, w4[q].y, w4[q].z, w4[q].w};
+        const uint32_t w[4] = {w4[r][q].x, w4[r][q].y, w4[r][q].z, w4[r][q].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           v[r][8 * q + 2 * i] = __uint_as_float(w[i] << 16);
           v[r][8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
       }
-    }
   }
+#pragma unroll
+  for (int r = 0; r < NR; ++r) nrm[r] = 1.f;
   if (ln) {
     // RMSNorm: sum of squares of the raw row; the gain per channel (on the
     // pass-0 layout with the transform, on the final layout without); the
@@ -509,13 +524,16 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
     const bool had = (flags & 1) != 0, int8 = (flags & 2) != 0, ln = (flags & 4) != 0;
     asm volatile("griddepcontrol.wait;\n" ::: "memory");   // X is ready past this point
     const float a_w = __ldg(alpha);
-    if (nr == 2) rows_phase<LOG_K, MT, 2>(X, m0, had, int8, ln, gain, xb, s_red, cbuf, meta);
-    else if (nr == 1) rows_phase<LOG_K, MT, 1>(X, m0, had, int8, ln, gain, xb, s_red, cbuf, meta);
+    // cluster barrier #1 (every peer runs and has armed its codes barrier) is
+    // waited while this CTA's X loads are in flight
+    const bool wait1 = csize > 1;
+    if (nr == 2) rows_phase<LOG_K, MT, 2>(X, m0, had, int8, ln, gain, xb, s_red, cbuf, meta, wait1);
+    else if (nr == 1) rows_phase<LOG_K, MT, 1>(X, m0, had, int8, ln, gain, xb, s_red, cbuf, meta, wait1);
+    else if (wait1) cluster_wait();
     fence_proxy_async_smem();   // the rows written here are read next by the bulk-copy engine
     consumers_sync();           // ... and by every consumer warp
     bool ok = true;
     if (csize > 1) {
-      cluster_wait();   // #1: every peer runs and has armed its codes barrier
       // lane 0 of warp w sends to peer w (warp 0 to peer csize - 1 ... all peers but this CTA)
       const uint32_t q = (uint32_t)warp;
       if (lane == 0 && nr > 0 && q < csize && q != crank) {
