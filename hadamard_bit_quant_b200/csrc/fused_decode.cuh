@@ -323,17 +323,18 @@ HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, bool had, boo
     mult = __fmul_rn(mult, nrm[r]);
     int csum = 0;
     uint32_t packed[E / 4];
+    if (int8) {
 #pragma unroll
-    for (int q = 0; q < E / 4; ++q) {
-      uint32_t w = 0u;
+      for (int q = 0; q < E / 4; ++q)
+        packed[q] = quant4<false>(v[r][4 * q], v[r][4 * q + 1], v[r][4 * q + 2], v[r][4 * q + 3], mult, 0.f, 0.f);
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = clampi(__float2int_rn(__fmul_rn(mult, v[r][4 * q + i])), lo, hi);
-        csum += c;
-        w |= ((uint32_t)(c & 0xff)) << (8 * i);
-      }
-      packed[q] = w;
+      for (int q = 0; q < E / 4; ++q)
+        packed[q] = quant4<true>(v[r][4 * q], v[r][4 * q + 1], v[r][4 * q + 2], v[r][4 * q + 3], mult, (float)lo,
+                                 (float)hi);
     }
+#pragma unroll
+    for (int q = 0; q < E / 4; ++q) csum = code_sum4(packed[q], csum);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) csum += __shfl_xor_sync(0xffffffffu, csum, off);
     if constexpr (E == 8) {

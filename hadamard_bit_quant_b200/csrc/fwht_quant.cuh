@@ -32,7 +32,11 @@ struct FwhtCfg {
   static constexpr int THREADS = T * TPC;
   static constexpr int P = (LOG_K + G - 1) / G;         // passes
   static constexpr int WARPS_PER_TOKEN = T >= 32 ? T / 32 : 1;
-  static constexpr int KPAD = K + K / E;                 // one pad word per E values
+  // Two-pass configurations whose token fills whole warps pad 4 words per E
+  // values (instead of 1), so the last pass reads its E consecutive values
+  // with 16-byte shared-memory loads, still free of bank conflicts.
+  static constexpr int PADW = (P == 2 && T >= 32) ? 4 : 1;
+  static constexpr int KPAD = K + PADW * (K / E);
   static constexpr size_t SMEM = (size_t)TPC * KPAD * sizeof(float);
 };
 
@@ -48,8 +52,37 @@ HBL_DEVINL int pass_index(int t, int j, int lo) {
 // index) the padded positions fall in 32 distinct banks, and because the
 // thread part and the register part of idx occupy disjoint bits, the
 // position splits into (thread part) + (compile-time offset per register).
-template <int G>
-HBL_DEVINL int pad(int idx) { return idx + (idx >> G); }
+template <int G, int PADW = 1>
+HBL_DEVINL int pad(int idx) { return idx + PADW * (idx >> G); }
+
+// Codes of four values, RoundClip(mult * v, lo, hi) with round half to even,
+// packed little-endian into one word. The product is rounded to fp32 first;
+// with CLAMP it is clamped to the integral bounds [lo, hi] (clamping commutes
+// with rounding to an integer there); adding 1.5 * 2^23 then rounds it to an
+// integer whose two's-complement low byte is the low mantissa byte of the sum
+// (|x| < 2^22). Without CLAMP the caller guarantees |mult * v| < 127.5 (the
+// absmax quantiser: |v| <= gamma < gamma + eps).
+template <bool CLAMP>
+HBL_DEVINL uint32_t quant4(float v0, float v1, float v2, float v3, float mult, float lo, float hi) {
+  const float2 m2 = make_float2(mult, mult);
+  float2 a = __fmul2_rn(make_float2(v0, v1), m2);
+  float2 b = __fmul2_rn(make_float2(v2, v3), m2);
+  if constexpr (CLAMP) {
+    a.x = fminf(fmaxf(a.x, lo), hi);
+    a.y = fminf(fmaxf(a.y, lo), hi);
+    b.x = fminf(fmaxf(b.x, lo), hi);
+    b.y = fminf(fmaxf(b.y, lo), hi);
+  }
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);
+  a = __fadd2_rn(a, magic);
+  b = __fadd2_rn(b, magic);
+  const uint32_t lo2 = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040);
+  const uint32_t hi2 = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040);
+  return __byte_perm(lo2, hi2, 0x5410);
+}
+
+// Sum of the four signed bytes of a packed code word, added to acc.
+HBL_DEVINL int code_sum4(uint32_t w, int acc) { return __dp4a((int)w, 0x01010101, acc); }
 
 // Sum / max over the T threads of one token. Threads of a token are T
 // consecutive lanes (T < 32) or T/32 whole warps (T >= 32). `red` holds one
@@ -146,14 +179,10 @@ HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool acti
     uint32_t packed[E / 4];
 #pragma unroll
     for (int q = 0; q < E / 4; ++q) {
-      uint32_t w = 0u;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = clampi(__float2int_rn(__fmul_rn(mult, v[4 * q + i])), lo, hi);
-        cs += c;
-        w |= ((uint32_t)(c & 0xff)) << (8 * i);
-      }
-      packed[q] = w;
+      packed[q] = MODE == kModeInt4
+                      ? quant4<true>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], mult, (float)lo, (float)hi)
+                      : quant4<false>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], mult, 0.f, 0.f);
+      cs = code_sum4(packed[q], cs);
     }
     if (csum != nullptr) cs = token_reduce_i<T, WPT>(cs, red_i, token_sub);   // uniform branch
     if (active) {
@@ -263,10 +292,20 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
       const int hi_prev = LOG_K - (p - 1) * G;
       const int lo_prev = hi_prev - G > 0 ? hi_prev - G : 0;
 #pragma unroll
-      for (int j = 0; j < E; ++j) sm[pad<G>(pass_index<G>(t, j, lo_prev))] = v[j];
+      for (int j = 0; j < E; ++j) sm[pad<G, C::PADW>(pass_index<G>(t, j, lo_prev))] = v[j];
       __syncthreads();
+      if (C::PADW == 4 && lo == 0) {
+        // last pass: E consecutive values at t * (E + 4), 16-byte aligned
+        const float4* src = reinterpret_cast<const float4*>(sm + t * (E + 4));
 #pragma unroll
-      for (int j = 0; j < E; ++j) v[j] = sm[pad<G>(pass_index<G>(t, j, lo))];
+        for (int q = 0; q < E / 4; ++q) {
+          const float4 f = src[q];
+          v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < E; ++j) v[j] = sm[pad<G, C::PADW>(pass_index<G>(t, j, lo))];
+      }
       if (p + 1 < P) __syncthreads();
     }
     butterflies<E>(v, nb);
@@ -368,18 +407,14 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const uint16_t* __rest
     scale = __fdiv_rn(r, 127.f);
     lo = -128; hi = 127;
   }
-  int cs = 0;
+  int cs = 0;   // inactive threads hold zeros, whose codes are 0
   uint32_t packed[E / 4];
 #pragma unroll
   for (int q = 0; q < E / 4; ++q) {
-    uint32_t w = 0u;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = clampi(__float2int_rn(__fmul_rn(mult, v[4 * q + i])), lo, hi);
-      cs += active ? c : 0;
-      w |= ((uint32_t)(c & 0xff)) << (8 * i);
-    }
-    packed[q] = w;
+    packed[q] = MODE == kModeInt4
+                    ? quant4<true>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], mult, (float)lo, (float)hi)
+                    : quant4<false>(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], mult, 0.f, 0.f);
+    cs = code_sum4(packed[q], cs);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) cs += __shfl_xor_sync(0xffffffffu, cs, off);
