@@ -11,7 +11,8 @@
 // codes; this kernel keeps every intermediate on chip:
 //   * one CTA per SM, grouped into clusters of CS CTAs (CS = 1, 2, 4 or 8);
 //   * a producer warp streams the weights of the CTA's 16-row groups through
-//     a TMA ring from the first instruction on, before the kernel waits for
+//     a TMA ring ([16 rows][64 B] boxes, one per 256-k block) from the first
+//     instruction on, before the kernel waits for
 //     the grid that produced X (programmatic dependent launch);
 //   * the 8 consumer warps of cluster rank r transform and quantise token rows
 //     2r and 2r + 1 (256 threads per row, E = K/256 values per thread,
@@ -47,7 +48,7 @@ constexpr int kConsumers = 8;
 constexpr int kRowThreads = 32 * kConsumers;        // threads per token row
 constexpr int kThreads = 32 * (kConsumers + 1);
 constexpr int kStages = 8;
-constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB = 4 boxes of [16][128 B]
+constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB = 8 boxes of [16][64 B], one per 256-k block
 constexpr int kMaxGroups = 8;
 constexpr int kRowBatch = 2;                        // token rows transformed together
 constexpr int kMaxTokens = 16;
@@ -92,6 +93,13 @@ HBL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, in
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
           su32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+HBL_DEVINL void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(
+          su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 HBL_DEVINL uint32_t cluster_rank() {
@@ -144,11 +152,14 @@ struct Layout {
 // Byte offset of the 16-byte code chunk holding k = 16*c16 .. 16*c16+15 of
 // token m: token rows are contiguous (K bytes each, so a row moves between
 // CTAs as one bulk copy); within each 128-byte segment the eight 16-byte
-// chunks are permuted by XOR with m % 8, which keeps the MMA fragment reads
-// (8 tokens x one chunk) free of bank conflicts.
+// chunks are permuted by XOR with 2 * (m % 4). An MMA fragment read (8-byte
+// loads) has each half-warp touch 4 tokens x 2 adjacent chunks; the
+// permutation puts those 8 (token, chunk) pairs on 8 distinct chunk slots, so
+// the read is free of bank conflicts.
+HBL_DEVINL int code_swz(int m) { return (m & 3) << 1; }
 template <int K>
 HBL_DEVINL uint32_t code_off(int m, int c16) {
-  return (uint32_t)(m * K + (c16 >> 3) * 128 + (((c16 & 7) ^ (m & 7)) << 4));
+  return (uint32_t)(m * K + (c16 >> 3) * 128 + (((c16 & 7) ^ code_swz(m)) << 4));
 }
 
 // Sum (or max) over the 256 consumer threads of NR values at once (one
@@ -365,7 +376,6 @@ HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, u
   constexpr int nchunks = K / kChunk;
   constexpr int SPLIT = TN == 1 ? 2 : 1;
   const int g = lane >> 2, tig = lane & 3;
-  const int ch = ((warp & 1) << 2) + tig;
   int acc[NG][TN * SPLIT][4];
 #pragma unroll
   for (int a = 0; a < NG; ++a)
@@ -382,7 +392,8 @@ HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, u
 #pragma unroll
       for (int i = 0; i < TN; ++i) {
         const int m = 8 * i + g;
-        bf[i][q] = *reinterpret_cast<const uint2*>(cbuf + m * K + box * 128 + ((cch ^ (m & 7)) << 4) + ((tig & 1) << 3));
+        bf[i][q] = *reinterpret_cast<const uint2*>(cbuf + m * K + box * 128 + ((cch ^ code_swz(m)) << 4) +
+                                                   ((tig & 1) << 3));
       }
     }
     uint32_t A4[NG][4], B4[NG][4];
@@ -391,9 +402,11 @@ HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, u
       const int u = c * NG + b;
       const int s = u % kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
-      const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
-      const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
-      const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+      // block `warp` of the unit: box `warp`, [16 rows][64 B]; rows sit 64 B
+      // apart, so the two rows a quarter-warp reads fall in different bank halves
+      const uint8_t* wb = ring + (size_t)s * kUnitBytes + warp * (kGroupRows * 64);
+      const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 64 + (tig << 4));
+      const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 64 + (tig << 4));
       A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
       B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
     }
@@ -438,7 +451,8 @@ HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, u
   return ok;
 }
 
-// flags: bit 0 use_hadamard, bit 1 INT8 (else INT4), bit 2 RMSNorm prologue.
+// flags: bit 0 use_hadamard, bit 1 INT8 (else INT4), bit 2 RMSNorm prologue,
+// bit 3 map_w is the 3-D blocked view (one copy per unit; else 2-D [16][64 B] boxes).
 template <int LOG_K, int TN>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* __restrict__ X, int M, int N,
@@ -465,6 +479,7 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
   const int Gd = gridDim.x;
   const int ng = (groups - (int)blockIdx.x + Gd - 1) / Gd;
   const int units = nchunks * ng;
+  const bool w3d = (flags & 8) != 0;
   // token rows [m0, m0 + nr) are transformed and quantised by this CTA
   const int m0 = (int)crank * kRowBatch;
   const int nr = M - m0 < 0 ? 0 : (M - m0 > kRowBatch ? kRowBatch : M - m0);
@@ -494,8 +509,13 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
       const int row0 = ((int)blockIdx.x + gl * Gd) * kGroupRows;
       mbar_expect_tx(&wfull[s], kUnitBytes);
       uint8_t* dst = ring + (size_t)s * kUnitBytes;
+      if (w3d) {
+        tma_load_3d(dst, &map_w, &wfull[s], 0, row0, c * (kChunk / kKBlock));   // 8 blocks x 16 rows x 64 B
+      } else {
 #pragma unroll
-      for (int b = 0; b < 4; ++b) tma_load_2d(dst + b * (kGroupRows * 128), &map_w, &wfull[s], c * (kChunk / 4) + b * 128, row0);
+        for (int b = 0; b < 8; ++b)
+          tma_load_2d(dst + b * (kGroupRows * 64), &map_w, &wfull[s], c * (kChunk / 4) + b * 64, row0);
+      }
     };
     if (lane == 0)
       for (; u < units && u < kStages; ++u) issue_w(u);

@@ -374,6 +374,23 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Packed weights viewed as [K/256 blocks][N rows][64 B] (block stride 64 B, row
+// stride K/4 B): one box of [8 blocks][16 rows][64 B] lands as eight
+// consecutive [16][64 B] tiles, the fused decode kernel's unit layout, in one
+// TMA copy.
+bool make_map_w_blocks(CUtensorMap* map, const void* Wpk, int N, int K) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)K / 256};
+  cuuint64_t strides[2] = {(cuuint64_t)K / 4, 64};
+  cuuint32_t box[3] = {64, 16, 8};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(Wpk), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D uint8 tensor map: rows x cols bytes, row stride `stride` bytes, box box_cols x box_rows.
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
                  uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
@@ -678,10 +695,16 @@ bool fused_fits(int M, int K, int N) {
 
 int run_fused_decode(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale, int act_bits,
                      int use_hadamard, bool ln, const float* gain, uint16_t* Y, int sm_count, cudaStream_t s) {
+  // [16 rows][64 B] tiles, unswizzled (the fused kernel's conflict-free fragment
+  // reads): one 3-D copy per 8 KB unit where the driver accepts the blocked
+  // view, else eight 2-D copies
   CUtensorMap mw;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, fdec::kGroupRows, true))
+  int flags = (use_hadamard ? 1 : 0) | (act_bits == 8 ? 2 : 0) | (ln ? 4 : 0);
+  if (make_map_w_blocks(&mw, Wpk, N, K)) {
+    flags |= 8;
+  } else if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 64, fdec::kGroupRows, false)) {
     return HBL_ERR_CUDA;
-  const int flags = (use_hadamard ? 1 : 0) | (act_bits == 8 ? 2 : 0) | (ln ? 4 : 0);
+  }
   const bool tn1 = M <= 8;
   switch (K) {
     case 2048: return tn1 ? launch_fused<11, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
