@@ -248,40 +248,78 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
                   float* __restrict__ scales, int32_t* __restrict__ csum, float* __restrict__ Xr) {
   using C = FwhtCfg<LOG_K, G>;
   constexpr int K = C::K, E = C::E, T = C::T, P = C::P;
-  extern __shared__ float smem[];
+  extern __shared__ __align__(16) float smem[];
   __shared__ float red_f[C::TPC * C::WARPS_PER_TOKEN];
   __shared__ int red_i[C::TPC * C::WARPS_PER_TOKEN];
+  __shared__ __align__(8) uint64_t stage_bar;
 
   const int token_sub = threadIdx.x / T;
   const int t = threadIdx.x % T;
   const size_t m = (size_t)blockIdx.x * C::TPC + token_sub;
   const bool active = m < (size_t)M;
   float* sm = smem + (size_t)token_sub * C::KPAD;
+  constexpr uint32_t kRowBytes = (uint32_t)K * (IN_F32 ? 4u : 2u);
+  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&stage_bar);
 
+  if (threadIdx.x == 0) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
+  __syncthreads();
   // Programmatic dependent launch: let the consumer grid launch now (it only
   // prefetches weights until this grid completes), and wait for the producer
   // of X before reading it. Both are no-ops without the launch attribute.
   asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  float v[E];
-  float ssq = 0.f;
-  // Pass 0 owns the top G bits: idx = t + j*T (coalesced across threads).
-  {
-    const size_t row = (active ? m : 0) * (size_t)K;
-#pragma unroll
-    for (int j = 0; j < E; ++j) {
-      float x = 0.f;
-      if (active) {
-        if constexpr (IN_F32) x = __ldg(reinterpret_cast<const float*>(Xv) + row + t + j * T);
-        else x = bf16_bits_to_float(__ldg(reinterpret_cast<const uint16_t*>(Xv) + row + t + j * T));
-      }
-      if constexpr (LN) {
-        ssq = __fmaf_rn(x, x, ssq);
-        if (gain) x = __fmul_rn(x, __ldg(gain + t + j * T));
-      }
-      v[j] = x;
+  // Each token's row arrives by one bulk copy into its exchange buffer; the
+  // first pass then reads its strided values (idx = t + j*T) from shared memory.
+  if (threadIdx.x == 0) {
+    const size_t m0 = (size_t)blockIdx.x * C::TPC;
+    const int n = (int)((size_t)M - m0 < (size_t)C::TPC ? (size_t)M - m0 : (size_t)C::TPC);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"((uint32_t)n * kRowBytes)
+                 : "memory");
+    for (int i = 0; i < n; ++i) {
+      const char* src = reinterpret_cast<const char*>(Xv) + (m0 + i) * (size_t)kRowBytes;
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(smem + (size_t)i * C::KPAD);
+      asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+                   "l"(src), "r"(kRowBytes), "r"(bar)
+                   : "memory");
     }
   }
+  {
+    uint32_t done = 0;
+    const long long t0 = clock64();
+    while (true) {
+      asm volatile("{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\nselp.u32 %0, 1, 0, p;\n}\n"
+                   : "=r"(done)
+                   : "r"(bar)
+                   : "memory");
+      if (done || clock64() - t0 > 4000000000ll) break;
+    }
+    if (!done && threadIdx.x == 0) set_device_error(HBL_ERR_TIMEOUT);
+  }
+  float v[E];
+  float ssq = 0.f;
+  // Pass 0 owns the top G bits: idx = t + j*T.
+  if (active) {
+    if constexpr (IN_F32) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) v[j] = sm[t + j * T];
+    } else {
+      const uint16_t* row = reinterpret_cast<const uint16_t*>(sm);
+#pragma unroll
+      for (int j = 0; j < E; ++j) v[j] = bf16_bits_to_float(row[t + j * T]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < E; ++j) v[j] = 0.f;
+  }
+  if constexpr (LN) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) ssq = __fmaf_rn(v[j], v[j], ssq);
+    if (gain) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) v[j] = __fmul_rn(v[j], __ldg(gain + t + j * T));
+    }
+  }
+  __syncthreads();   // the staged rows are consumed; the exchanges overwrite them
 #pragma unroll
   for (int p = 0; p < P; ++p) {
     const int hi = LOG_K - p * G;
