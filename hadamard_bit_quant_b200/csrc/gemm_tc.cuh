@@ -9,7 +9,7 @@
 // (u = t + 1 in {0,1,2}; the exact product is D - sum_k c):
 //   * warp 0 (one lane): TMA producer. Per 256-k stage it loads the codes
 //     tile (256 tokens x 256 k, two 128-byte-wide boxes, 128B swizzle) and the
-//     packed weight tile (128 rows x 64 bytes).
+//     packed weight tile (128 rows x 64 bytes, 64B swizzle).
 //   * warps 2..5: converters. Each thread owns one weight row (one TMEM lane),
 //     unpacks its 64 packed bytes into 256 unsigned bytes in registers and
 //     writes them into the stage's 64 TMEM columns with tcgen05.st. The
@@ -248,11 +248,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
       const int s = kb % kStages;
       const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], ph, abort))) break;
+      // the tile arrives 64B-swizzled: 16-byte chunk t of row `row` sits at
+      // chunk t ^ ((row >> 1) & 3), which spreads a quarter-warp's 8 rows over
+      // all 32 banks
       const uint4* src = reinterpret_cast<const uint4*>(&S.a[s][row * (kKBlock / 4)]);
       uint32_t wv[16];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const uint4 q = src[t];
+        const uint4 q = src[t ^ ((row >> 1) & 3)];
         wv[4 * t] = q.x; wv[4 * t + 1] = q.y; wv[4 * t + 2] = q.z; wv[4 * t + 3] = q.w;
       }
       // word (tig, w) register j holds k = 64w + 32(j>>1) + 8tig + 4(j&1) + i, i.e.

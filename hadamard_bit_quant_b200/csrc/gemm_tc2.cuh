@@ -191,11 +191,12 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_cons
         const int s = g % kStages;
         const uint32_t ph = (uint32_t)(g / kStages) & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], ph, abort))) { ok = false; break; }
+        // 64B-swizzled tile: chunk q of the row sits at q ^ ((row >> 1) & 3)
         const uint4* src = reinterpret_cast<const uint4*>(&S.a[s][row * (kKBlock / 4)]);
         uint32_t wv[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint4 v = src[q];
+          const uint4 v = src[q ^ ((row >> 1) & 3)];
           wv[4 * q] = v.x; wv[4 * q + 1] = v.y; wv[4 * q + 2] = v.z; wv[4 * q + 3] = v.w;
         }
         uint32_t c0[32], c1[32];

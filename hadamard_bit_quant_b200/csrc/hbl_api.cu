@@ -391,9 +391,10 @@ bool make_map_w_blocks(CUtensorMap* map, const void* Wpk, int N, int K) {
   return r == CUDA_SUCCESS;
 }
 
-// 2-D uint8 tensor map: rows x cols bytes, row stride `stride` bytes, box box_cols x box_rows.
+// 2-D uint8 tensor map: rows x cols bytes, row stride `stride` bytes, box box_cols x box_rows,
+// swizzle_bytes 0 (none), 64 or 128.
 bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t stride,
-                 uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+                 uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -401,7 +402,9 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : (swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -418,8 +421,8 @@ int run_gemm_tc2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, c
                  const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count,
                  cudaStream_t s) {
   CUtensorMap mc, mw;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc2::kToks, true)) return HBL_ERR_CUDA;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc2::kRows, false))
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc2::kToks, 128)) return HBL_ERR_CUDA;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc2::kRows, 64))
     return HBL_ERR_CUDA;
   const int tiles = ((N + tc2::kRows - 1) / tc2::kRows) * ((M + tc2::kToks - 1) / tc2::kToks);
   const dim3 grid(tiles < sm_count ? tiles : sm_count);
@@ -440,8 +443,8 @@ int run_gemm_tc2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, c
 int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
                 const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
   CUtensorMap mc, mw;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc::kToks, true)) return HBL_ERR_CUDA;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc::kRows, false))
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc::kToks, 128)) return HBL_ERR_CUDA;
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc::kRows, 64))
     return HBL_ERR_CUDA;
   dim3 grid((N + tc::kRows - 1) / tc::kRows, (M + tc::kToks - 1) / tc::kToks);
   ProfScope ps("gemm_tc", s);
@@ -518,9 +521,9 @@ int run_gemm_decode2(const int8_t* codes, int M, int K, int N, const uint8_t* Wp
   if (!decode2_config(M, K, &C, &KC, &smem)) return HBL_ERR_UNSUPPORTED;
   const int TN = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
   CUtensorMap mw, mc;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, dec2::kRows, true))
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, dec2::kRows, 128))
     return HBL_ERR_CUDA;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), true))
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), 128))
     return HBL_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, (N + dec2::kRows - 1) / dec2::kRows);
@@ -571,9 +574,9 @@ int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
                     cudaStream_t s) {
   const int TN = M <= 8 ? 1 : 2;
   CUtensorMap mw, mc;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, strm::kGroupRows, true))
+  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, strm::kGroupRows, 128))
     return HBL_ERR_CUDA;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), true))
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), 128))
     return HBL_ERR_CUDA;
   const int groups = N / strm::kGroupRows;
   const dim3 grid(groups < sm_count ? groups : sm_count);
@@ -702,7 +705,7 @@ int run_fused_decode(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk,
   int flags = (use_hadamard ? 1 : 0) | (act_bits == 8 ? 2 : 0) | (ln ? 4 : 0);
   if (make_map_w_blocks(&mw, Wpk, N, K)) {
     flags |= 8;
-  } else if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 64, fdec::kGroupRows, false)) {
+  } else if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 64, fdec::kGroupRows, 0)) {
     return HBL_ERR_CUDA;
   }
   const bool tn1 = M <= 8;
