@@ -5,10 +5,10 @@
 // Layer", Eq. 9: acc[m, n] = sum_k c[m, k] * t[n, k], then the dequant
 // acc * s[m] * alpha (Eq. 1, Eq. 7 / Eq. 8).
 //
-// One CTA computes a 128 (output features) x 256 (tokens) tile of D = sum c*u
+// One CTA computes a 128 (output features) x TOKS (tokens: 128, 192 or 256) tile of D = sum c*u
 // (u = t + 1 in {0,1,2}; the exact product is D - sum_k c):
 //   * warp 0 (one lane): TMA producer. Per 256-k stage it loads the codes
-//     tile (256 tokens x 256 k, two 128-byte-wide boxes, 128B swizzle) and the
+//     tile (TOKS tokens x 256 k, two 128-byte-wide boxes, 128B swizzle) and the
 //     packed weight tile (128 rows x 64 bytes, 64B swizzle).
 //   * warps 2..5: converters. Each thread owns one weight row (one TMEM lane),
 //     unpacks its 64 packed bytes into 256 unsigned bytes in registers and
@@ -16,8 +16,8 @@
 //     weights thus become the MMA's A operand straight from tensor memory and
 //     never pass through shared memory unpacked.
 //   * warp 1 (one lane): MMA issuer. Eight tcgen05.mma.kind::i8 (M=128,
-//     N=256, K=32) per stage, A from TMEM, B (codes) from shared memory,
-//     int32 accumulator in TMEM columns [0, 256); tcgen05.commit frees the stage.
+//     N=TOKS, K=32) per stage, A from TMEM, B (codes) from shared memory,
+//     int32 accumulator in TMEM columns [0, TOKS); tcgen05.commit frees the stage.
 //   * warps 2..5 again: epilogue. tcgen05.ld of the accumulator, subtract the
 //     code sum, scale by s[m] * alpha, store bf16 (or the int32 result).
 // Every mbarrier wait is bounded (about a second of clock cycles); on timeout
@@ -31,28 +31,37 @@ namespace hbl {
 namespace tc {
 
 constexpr int kRows = 128;         // weight rows per tile (MMA M)
-constexpr int kToks = 256;         // tokens per tile (MMA N)
 constexpr int kStages = 3;
-constexpr int kBBytes = kToks * kKBlock;          // 64 KB codes per stage
 constexpr int kABytes = kRows * (kKBlock / 4);    // 8 KB packed weights per stage
-constexpr int kStageTx = kBBytes + kABytes;
-constexpr int kDCols = kToks;                     // accumulator columns
 constexpr int kACols = kKBlock / 4;               // 64 TMEM columns of A per stage
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr long long kSpinLimit = 4000000000ll;    // ~2 s of SM clock
 
-struct __align__(8) Smem {
-  uint8_t b[kStages][kBBytes];      // 1024-byte aligned (swizzle atoms)
-  uint8_t a[kStages][kABytes];
-  uint64_t full[kStages];
-  uint64_t aready[kStages];
-  uint64_t empty[kStages];
-  uint64_t done;
-  uint32_t tmem_base;
-  int abort;
+// TOKS tokens per tile (the MMA's N, a multiple of 64 from 128 to 256; the
+// launcher uses 256).
+template <int TOKS>
+struct Tile {
+  static_assert(TOKS % 64 == 0 && TOKS >= 128 && TOKS <= 256, "token tile");
+  static constexpr int kBBytes = TOKS * kKBlock;          // codes per stage (two [TOKS][128 B] boxes)
+  static constexpr int kStageTx = kBBytes + kABytes;
+  static constexpr int kDCols = TOKS;                     // accumulator columns
+  static_assert(kDCols + kStages * kACols <= kTmemCols, "TMEM columns");
+  struct __align__(8) Smem {
+    uint8_t b[kStages][kBBytes];      // 1024-byte aligned (swizzle atoms)
+    uint8_t a[kStages][kABytes];
+    uint64_t full[kStages];
+    uint64_t aready[kStages];
+    uint64_t empty[kStages];
+    uint64_t done;
+    uint32_t tmem_base;
+    int abort;
+  };
+  static constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+  // Instruction descriptor: D s32, A u8, B s8, both K-major, M = 128, N = TOKS.
+  static constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(TOKS >> 3) << 17) |
+                                     ((uint32_t)(kRows >> 4) << 24);
 };
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
 
 HBL_DEVINL uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -124,9 +133,6 @@ HBL_DEVINL void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uin
       : "memory");
 }
 
-// Instruction descriptor: D s32, A u8, B s8, both K-major, M = 128, N = 256.
-constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(kToks >> 3) << 17) |
-                            ((uint32_t)(kRows >> 4) << 24);
 
 // Shared-memory descriptor of a K-major, 128B-swizzled tile whose rows are
 // 128 bytes and whose 8-row groups are 1024 bytes apart.
@@ -162,16 +168,20 @@ HBL_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
       : "memory")
 
 // OUT_BF16: Y = bf16((D - csum) * s * alpha); else acc (int32) = D - csum.
-template <bool OUT_BF16>
+template <bool OUT_BF16, int TOKS>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_w, int M,
                int K, int N, const int32_t* __restrict__ csum, const float* __restrict__ scales,
                const float* __restrict__ alpha, uint16_t* __restrict__ Y, int32_t* __restrict__ acc_out) {
+  using TL = Tile<TOKS>;
+  using Smem = typename TL::Smem;
+  constexpr int kBBytes = TL::kBBytes, kStageTx = TL::kStageTx, kDCols = TL::kDCols;
+  constexpr uint32_t kIdesc = TL::kIdesc;
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kRows;
-  const int m0 = blockIdx.y * kToks;
+  const int m0 = blockIdx.y * TOKS;
   const int nblk = K / kKBlock;
   volatile int* abort = &S.abort;
 

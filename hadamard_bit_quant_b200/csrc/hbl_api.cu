@@ -128,8 +128,6 @@ int ensure_device(DeviceState** out) {
         cudaFuncSetAttribute(dec::gemm_decode_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
         cudaFuncSetAttribute(dec::gemm_decode_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
       }
-      cudaFuncSetAttribute(tc::gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
-      cudaFuncSetAttribute(tc::gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
       if (cudaGetLastError() != cudaSuccess) return HBL_ERR_CUDA;
     }
   }
@@ -440,21 +438,37 @@ int run_gemm_tc2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, c
 }
 
 // bf16 output (Y != nullptr) or int32 output (acc != nullptr); D - csum either way.
+template <int TOKS>
+int launch_gemm_tc(const CUtensorMap& mc, const CUtensorMap& mw, int M, int K, int N, const int32_t* csum,
+                   const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
+  using TL = tc::Tile<TOKS>;
+  const dim3 grid((N + tc::kRows - 1) / tc::kRows, (M + TOKS - 1) / TOKS);
+  ProfScope ps("gemm_tc", s);
+  if (Y) {
+    ensure_smem_attr(tc::gemm_tc_kernel<true, TOKS>, TL::kSmemBytes);
+    tc::gemm_tc_kernel<true, TOKS><<<grid, tc::kThreads, TL::kSmemBytes, s>>>(mc, mw, M, K, N, csum, scales, alpha,
+                                                                               Y, nullptr);
+  } else {
+    ensure_smem_attr(tc::gemm_tc_kernel<false, TOKS>, TL::kSmemBytes);
+    tc::gemm_tc_kernel<false, TOKS><<<grid, tc::kThreads, TL::kSmemBytes, s>>>(mc, mw, M, K, N, csum, nullptr,
+                                                                                nullptr, nullptr, acc);
+  }
+  return launch_status();
+}
+
+// One-tile-per-CTA tcgen05 GEMM with 128 x 256 tiles. (Measured on B200 over
+// prefill shapes, 256-token tiles beat 192 and 128 everywhere even where
+// narrower tiles fill the last wave better: the kernel is bound by feeding
+// codes from L2, and a wider tile re-reads the weights less.)
 int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
-                const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
+                const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count, cudaStream_t s) {
+  (void)sm_count;
+  constexpr int toks = 256;
   CUtensorMap mc, mw;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tc::kToks, 128)) return HBL_ERR_CUDA;
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)toks, 128)) return HBL_ERR_CUDA;
   if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc::kRows, 64))
     return HBL_ERR_CUDA;
-  dim3 grid((N + tc::kRows - 1) / tc::kRows, (M + tc::kToks - 1) / tc::kToks);
-  ProfScope ps("gemm_tc", s);
-  if (Y)
-    tc::gemm_tc_kernel<true><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(mc, mw, M, K, N, csum, scales, alpha, Y,
-                                                                        nullptr);
-  else
-    tc::gemm_tc_kernel<false><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(mc, mw, M, K, N, csum, nullptr, nullptr,
-                                                                         nullptr, acc);
-  return launch_status();
+  return launch_gemm_tc<toks>(mc, mw, M, K, N, csum, scales, alpha, Y, acc, s);
 }
 
 bool decode_path_fits(int M, int K) {
@@ -738,7 +752,7 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   if (st) return st;
   switch (choose_gemm(M, K, N)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
-    case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s);
+    case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
     case GemmKind::Decode: return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count);
     case GemmKind::Mma: break;
   }
@@ -920,7 +934,7 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   if ((st = launch_status())) return st;
   switch (choose_gemm(M, K, N)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
-    case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s);
+    case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
     case GemmKind::Decode: return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count);
     case GemmKind::Mma: break;
   }
