@@ -355,6 +355,88 @@ def secondary(torch, hbl, layer, inputs):
     return out
 
 
+def _event_ms(torch, fn, reps=5, flush=None):
+    """Median CUDA-event time (ms) of fn(), L2 flushed before each run."""
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def next_rows(torch, hbl, layer, inputs, peak_gbs):
+    """The next rows beyond the forward: RMSNorm prologue (f1), rotated-weight packing (f2),
+    Hadamard backward (f3), post-RoPE QKV quantiser (f4). Bytes per call are algorithmic
+    (what the kernel must read and write); all are bound by HBM."""
+    out = {}
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    g = torch.Generator().manual_seed(7)
+
+    def rec(name, ms, nbytes, **extra):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"us": ms * 1e3, "bytes": nbytes, "GBps": gbs, "frac_of_hbm": gbs / peak_gbs, **extra}
+
+    # f1: RMSNorm + Hadamard + INT4 quantiser, prefill-sized
+    M, K = 4096, 16384
+    X = (torch.randn(M, K, generator=g)).to(torch.bfloat16).cuda()
+    gain = (0.5 + torch.rand(K, generator=g)).cuda()
+    codes = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    sc = torch.empty(M, device="cuda")
+    cs = torch.empty(M, dtype=torch.int32, device="cuda")
+    ms = _event_ms(torch, lambda: hbl.hbl_quantize_ln(X, M, K, gain, 4, 1, codes, sc, cs), flush=flush)
+    rec("f1 quantize_ln M=4096 K=16384 A4 H on", ms, M * (2 * K + K + 8) + 4 * K)
+    # f1: the whole forward with the prologue, decode o_proj shape (fused kernel), 64 weight sets
+    case = [c for c in inputs.decode_oproj_cases((HEAD["M"],), (HEAD["act_bits"],))][0]
+    Xd = case.make_x().cuda()
+    gd = (0.5 + torch.rand(case.K, generator=g)).cuda()
+    Wpk, wsc = layer.pack_weights(case.make_w().cuda())
+    Wpks = [Wpk] + [Wpk.clone() for _ in range(LAYERS - 1)]
+    Y = torch.empty(case.M, case.N, dtype=torch.bfloat16, device="cuda")
+    ws = layer.workspace(case.M, case.K, case.N, "cuda")
+    hbl.hbl_forward_ln_ws(Xd, case.M, case.K, case.N, gd, Wpk, wsc, case.act_bits, 1, Y, ws, ws.numel())
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    with torch.cuda.graph(graph, stream=st):
+        for w in Wpks:
+            hbl.hbl_forward_ln_ws(Xd, case.M, case.K, case.N, gd, w, wsc, case.act_bits, 1, Y, ws, ws.numel(),
+                                  torch.cuda.current_stream().cuda_stream)
+    ms = timed_replays(torch, None, graph, 3, 20, 1) / (20 * LAYERS)
+    rec(f"f1 forward_ln decode M={case.M} K={case.K} N={case.N} A{case.act_bits}", ms,
+        case.N * case.K // 4 + 2 * case.M * case.K + 2 * case.M * case.N + 4 * case.K + 4,
+        tokens_per_s=case.M / (ms * 1e-3))
+    del graph, Wpks
+    # f2: rotated-weight packing (offline), 4096 x 4096
+    N2 = K2 = 4096
+    W = (0.02 * torch.randn(N2, K2, generator=g)).cuda()
+    Wpk2 = torch.empty(hbl.hbl_packed_bytes(N2, K2), dtype=torch.uint8, device="cuda")
+    a2 = torch.empty(1, device="cuda")
+    Wrot = torch.empty(N2, K2, device="cuda")
+    ms = _event_ms(torch, lambda: hbl.hbl_pack_weights_rotated(W, N2, K2, Wpk2, a2, Wrot), flush=flush)
+    rec("f2 pack_weights_rotated N=K=4096", ms, 4 * N2 * K2 + 4 * N2 * K2 + N2 * K2 // 4)
+    # f3: Hadamard backward, fp32 gradients, prefill-sized
+    dXr = torch.randn(M, K, generator=g).cuda()
+    dX = torch.empty_like(dXr)
+    ms = _event_ms(torch, lambda: hbl.hbl_hadamard_backward_f32(dXr, M, K, dX), flush=flush)
+    rec("f3 hadamard_backward_f32 M=4096 K=16384", ms, 8 * M * K)
+    del dXr, dX
+    # f4: post-RoPE QKV quantiser, 4 bits, BOS at 8 bits
+    T, H, d = 4096, 32, 128
+    Xq = torch.randn(T, H, d, generator=g).to(torch.bfloat16).cuda()
+    cq = torch.empty(T, H, d, dtype=torch.uint8, device="cuda")
+    gq = torch.empty(T, H, device="cuda")
+    ms = _event_ms(torch, lambda: hbl.hbl_quantize_qkv(Xq, T, H, d, 4, 0, cq, gq), flush=flush)
+    rec("f4 quantize_qkv T=4096 H=32 d=128 4-bit", ms, 2 * T * H * d + T * H * d + 4 * T * H)
+    return out
+
+
 def run_ours(args, rank, world, local):
     import torch
     import torch.distributed as dist
@@ -423,6 +505,10 @@ def run_ours(args, rank, world, local):
             line["secondary"] = secondary(torch, hbl, layer, inputs)
         except Exception as ex:  # secondary numbers are optional context
             line["secondary"] = {"error": repr(ex)}
+        try:
+            line["next_rows"] = next_rows(torch, hbl, layer, inputs, peaks["hbm_gbs"])
+        except Exception as ex:
+            line["next_rows"] = {"error": repr(ex)}
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_oracle_baseline(Xc, Wc, c)
     if rank == 0:
