@@ -1009,7 +1009,8 @@ int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_t
   if (st) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int rows = T * H;
-  const dim3 grid((rows + 7) / 8);
+  const int per_cta = 8 * kQkvRowsPerWarp;
+  const dim3 grid((rows + per_cta - 1) / per_cta);
   ProfScope ps("qkv_quant", s);
   if (d == 64) qkv_quant_kernel<2><<<grid, 256, 0, s>>>(X, rows, H, bits, bos_token, codes, gamma);
   else if (d == 128) qkv_quant_kernel<4><<<grid, 256, 0, s>>>(X, rows, H, bits, bos_token, codes, gamma);
