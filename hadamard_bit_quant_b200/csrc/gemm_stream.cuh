@@ -9,15 +9,16 @@
 //   * one CTA per SM (persistent); CTA c owns the 16-row groups c, c+G, ...
 //     over the whole of K, so no partial sums ever leave the CTA;
 //   * K is walked in chunks of 2048; a chunk's codes (M x 2048 int8) sit in
-//     one of two shared-memory buffers, loaded once per chunk by TMA;
+//     one of two shared-memory buffers, one bulk copy per token row;
 //   * the weights of each (chunk, group) unit -- 16 rows x 512 bytes -- stream
-//     through a 16-stage TMA ring (128 KB in flight per SM). The ring is
+//     through a 16-stage ring (128 KB in flight per SM), one 3-D TMA copy per
+//     unit laid out as eight [16 rows][64 B] tiles. The ring is
 //     filled before the kernel waits for the quantiser grid (programmatic
 //     dependent launch), so a layer's weights arrive while the previous
 //     kernel still runs;
 //   * 8 consumer warps take one 256-k block of each unit each: weights as the
 //     m16n8k32 A operand (u = t + 1 unpacked in registers), codes as B, both
-//     from 128B-swizzled shared memory (conflict-free), accumulating in
+//     read free of bank conflicts, accumulating in
 //     registers across chunks; a dedicated producer warp issues the copies;
 //   * at the end the 8 warps' partial sums are added in shared memory, the
 //     code sums subtracted, scaled and stored as bf16 (or int32).
@@ -75,6 +76,20 @@ HBL_DEVINL bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
   }
   return true;
 }
+HBL_DEVINL void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(
+          su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// Contiguous global -> shared copy of `bytes` (multiple of 16, both ends 16-byte aligned).
+HBL_DEVINL void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   su32(dst)),
+               "l"(src), "r"(bytes), "r"(su32(bar))
+               : "memory");
+}
 HBL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
@@ -83,10 +98,14 @@ HBL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, in
       : "memory");
 }
 
+// One chunk of codes: MT token rows of kChunk bytes, row stride kChunk + 32
+// (each token row arrives by one bulk copy). The 32-byte pad puts rows m and
+// m + 1 four banks apart, so an m16n8k32 fragment read (each half-warp: 4
+// tokens x 32 bytes) touches 16 distinct 8-byte bank slots.
 template <int MT>
 struct Layout {
-  static constexpr int kCodeBox = MT * 128;                 // one [MT][128 B] box
-  static constexpr int kCodeBuf = (kChunk / 128) * kCodeBox;
+  static constexpr int kCodeRow = kChunk + 32;
+  static constexpr int kCodeBuf = MT * kCodeRow;
   static constexpr size_t kRing = (size_t)kStages * kUnitBytes;
   static constexpr size_t kBytes = 1024 + kRing + 2 * (size_t)kCodeBuf + 256;
 };
@@ -103,7 +122,6 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
   using Lay = Layout<MT>;
   constexpr int SPLIT = TN == 1 ? 2 : 1;
   const int g = lane >> 2, tig = lane & 3;
-  const int ch = ((warp & 1) << 2) + tig;
   int acc[NG][TN * SPLIT][4];
 #pragma unroll
   for (int a = 0; a < NG; ++a)
@@ -118,12 +136,10 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
     uint2 bf[TN][8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const int box = 2 * warp + (q >> 2), cch = 2 * (q & 3) + (tig >> 1);
 #pragma unroll
       for (int i = 0; i < TN; ++i) {
-        const int m = 8 * i + g;
-        bf[i][q] = *reinterpret_cast<const uint2*>(cb + box * Lay::kCodeBox + m * 128 + ((cch ^ (m & 7)) << 4) +
-                                                   ((tig & 1) << 3));
+        const int m = 8 * i + g;   // k = 256 * warp + 32 * q + 8 * tig .. + 7 of the chunk
+        bf[i][q] = *reinterpret_cast<const uint2*>(cb + m * Lay::kCodeRow + 256 * warp + 32 * q + 8 * tig);
       }
     }
     __syncwarp();
@@ -134,9 +150,11 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
       const int u = c * NG + b;
       const int s = u % kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
-      const uint8_t* wb = ring + (size_t)s * kUnitBytes + (warp >> 1) * (kGroupRows * 128);
-      const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 128 + ((ch ^ g) << 4));
-      const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 128 + ((ch ^ g) << 4));
+      // block `warp` of the unit: tile `warp`, [16 rows][64 B]; rows 64 B apart,
+      // so the two rows a quarter-warp reads fall in different bank halves
+      const uint8_t* wb = ring + (size_t)s * kUnitBytes + warp * (kGroupRows * 64);
+      const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 64 + (tig << 4));
+      const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 64 + (tig << 4));
       A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
       B4[b][0] = pb.x; B4[b][1] = pb.y; B4[b][2] = pb.z; B4[b][3] = pb.w;
     }
@@ -185,7 +203,7 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
 
 template <int TN, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_c,
+gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __restrict__ codes,
                    const int32_t* __restrict__ csum, const float* __restrict__ scales,
                    const float* __restrict__ alpha, int M, int K, int N, uint16_t* __restrict__ Y,
                    int32_t* __restrict__ acc_out) {
@@ -231,14 +249,14 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_const
         const int c = u / ng, gl = u % ng;
         const int row0 = ((int)blockIdx.x + gl * G) * kGroupRows;
         mbar_expect_tx(&wfull[s], kUnitBytes);
-        uint8_t* dst = ring + (size_t)s * kUnitBytes;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) tma_load_2d(dst + b * (kGroupRows * 128), &map_w, &wfull[s], c * (kChunk / 4) + b * 128, row0);
+        // 8 blocks x 16 rows x 64 B: eight [16][64 B] tiles in one copy
+        tma_load_3d(ring + (size_t)s * kUnitBytes, &map_w, &wfull[s], 0, row0, c * (kChunk / kKBlock));
       };
       auto issue_c = [&](int c) {
         uint8_t* dst = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
-        mbar_expect_tx(&cfull[c & 1], (uint32_t)Lay::kCodeBuf);
-        for (int b = 0; b < kChunk / 128; ++b) tma_load_2d(dst + b * Lay::kCodeBox, &map_c, &cfull[c & 1], c * kChunk + b * 128, 0);
+        mbar_expect_tx(&cfull[c & 1], (uint32_t)(M * kChunk));
+        for (int m = 0; m < M; ++m)
+          bulk_load(dst + m * Lay::kCodeRow, codes + (size_t)m * K + (size_t)c * kChunk, kChunk, &cfull[c & 1]);
       };
       int u = 0;
       for (; u < units && u < kStages; ++u) issue_w(u);             // weights do not depend on the previous grid

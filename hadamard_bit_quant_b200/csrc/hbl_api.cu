@@ -583,15 +583,13 @@ bool stream_fits(int M, int K, int N, int sm_count) {
   return G > 0 && groups <= strm::kMaxGroups * G;
 }
 
+// -1: the blocked weight view could not be encoded; the caller takes another decode kernel.
 int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
                     const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count,
                     cudaStream_t s) {
   const int TN = M <= 8 ? 1 : 2;
-  CUtensorMap mw, mc;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, 128, strm::kGroupRows, 128))
-    return HBL_ERR_CUDA;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)(8 * TN), 128))
-    return HBL_ERR_CUDA;
+  CUtensorMap mw;
+  if (!make_map_w_blocks(&mw, Wpk, N, K)) return -1;
   const int groups = N / strm::kGroupRows;
   const dim3 grid(groups < sm_count ? groups : sm_count);
   ProfScope ps("gemm_decode", s);
@@ -601,11 +599,11 @@ int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
     const size_t sm = strm::Layout<8 * TN_>::kBytes;                                                           \
     if (Y) {                                                                                                   \
       ensure_smem_attr(strm::gemm_stream_kernel<TN_, true>, sm);                                               \
-      e = launch_pdl(strm::gemm_stream_kernel<TN_, true>, grid, dim3(strm::kThreads), sm, s, mw, mc, csum,      \
+      e = launch_pdl(strm::gemm_stream_kernel<TN_, true>, grid, dim3(strm::kThreads), sm, s, mw, codes, csum,   \
                      scales, alpha, M, K, N, Y, (int32_t*)nullptr);                                            \
     } else {                                                                                                   \
       ensure_smem_attr(strm::gemm_stream_kernel<TN_, false>, sm);                                              \
-      e = launch_pdl(strm::gemm_stream_kernel<TN_, false>, grid, dim3(strm::kThreads), sm, s, mw, mc, csum,     \
+      e = launch_pdl(strm::gemm_stream_kernel<TN_, false>, grid, dim3(strm::kThreads), sm, s, mw, codes, csum,  \
                      (const float*)nullptr, (const float*)nullptr, M, K, N, (uint16_t*)nullptr, acc);          \
     }                                                                                                          \
   }
@@ -617,8 +615,10 @@ int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
                     const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s,
                     int sm_count = 148) {
-  if ((g_gemm_path == 0 || g_gemm_path == 5) && stream_fits(M, K, N, sm_count))
-    return run_gemm_stream(codes, M, K, N, Wpk, csum, scales, alpha, Y, acc, sm_count, s);
+  if ((g_gemm_path == 0 || g_gemm_path == 5 || g_gemm_path == 6) && stream_fits(M, K, N, sm_count)) {
+    const int st = run_gemm_stream(codes, M, K, N, Wpk, csum, scales, alpha, Y, acc, sm_count, s);
+    if (st >= 0) return st;
+  }
   {
     int C, KC;
     size_t sm;
