@@ -64,6 +64,16 @@ HBL_DEVINL bool mbar_try_wait(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking probe (test_wait never suspends the thread).
+HBL_DEVINL bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 HBL_DEVINL bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort) {
   const long long t0 = clock64();
   while (!mbar_try_wait(b, parity)) {
@@ -107,14 +117,18 @@ struct Layout {
   static constexpr int kCodeRow = kChunk + 32;
   static constexpr int kCodeBuf = MT * kCodeRow;
   static constexpr size_t kRing = (size_t)kStages * kUnitBytes;
-  static constexpr size_t kBytes = 1024 + kRing + 2 * (size_t)kCodeBuf + 256;
+  // wfull, wempty [kStages]; cfull, cempty [2]; abort flag
+  static constexpr size_t kBarBytes = (size_t)(2 * kStages + 4) * 8 + 16;
+  static constexpr size_t kBytes = 1024 + kRing + 2 * (size_t)kCodeBuf + kBarBytes;
 };
 
 // Consumer side for a CTA that owns exactly NG groups: per chunk, wait for
 // the chunk's codes and all NG weight units, load every fragment, release the
 // slots, then issue the chunk's MMAs q by q over all groups (2*NG independent
 // accumulator chains; with one token tile, even and odd q accumulate
-// separately). Ends by writing this warp's partial sums into shared memory
+// separately). The NG unit barriers are probed back to back with test_wait
+// (non-blocking), so their round trips (on the order of a hundred cycles
+// each) overlap; only a unit still in flight is waited for. Ends by writing this warp's partial sums into shared memory
 // (aliasing the ring) once every consumer warp is past its last unit.
 template <int NG, int TN, int MT>
 HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, uint64_t* wempty,
@@ -145,11 +159,17 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
     __syncwarp();
     if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
     uint32_t A4[NG][4], B4[NG][4];
+    bool landed[NG];
+#pragma unroll
+    for (int b = 0; b < NG; ++b) {
+      const int u = c * NG + b;
+      landed[b] = mbar_test(&wfull[u % kStages], (uint32_t)(u / kStages) & 1u);
+    }
 #pragma unroll
     for (int b = 0; b < NG; ++b) {
       const int u = c * NG + b;
       const int s = u % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
+      if (!__all_sync(0xffffffffu, landed[b] || mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
       // block `warp` of the unit: tile `warp`, [16 rows][64 B]; rows 64 B apart,
       // so the two rows a quarter-warp reads fall in different bank halves
       const uint8_t* wb = ring + (size_t)s * kUnitBytes + warp * (kGroupRows * 64);
