@@ -480,9 +480,11 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
   const int ng = (groups - (int)blockIdx.x + Gd - 1) / Gd;
   const int units = nchunks * ng;
   const bool w3d = (flags & 8) != 0;
-  // token rows [m0, m0 + nr) are transformed and quantised by this CTA
-  const int m0 = (int)crank * kRowBatch;
-  const int nr = M - m0 < 0 ? 0 : (M - m0 > kRowBatch ? kRowBatch : M - m0);
+  // token rows [m0, m0 + nr) are transformed and quantised by this CTA:
+  // ceil(M / cluster size) rows each (at most kRowBatch, checked at launch)
+  const int rpc = (M + (int)csize - 1) / (int)csize;
+  const int m0 = (int)crank * rpc;
+  const int nr = M - m0 < 0 ? 0 : (M - m0 > rpc ? rpc : M - m0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -555,14 +557,16 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
     consumers_sync();           // ... and by every consumer warp
     bool ok = true;
     if (csize > 1) {
-      // lane 0 of warp w sends to peer w (warp 0 to peer csize - 1 ... all peers but this CTA)
-      const uint32_t q = (uint32_t)warp;
-      if (lane == 0 && nr > 0 && q < csize && q != crank) {
-        const uint32_t bar = map_rank(su32(codes_full), q);
-        const uint32_t cb_off = (uint32_t)m0 * Lay::K, mt_off = (uint32_t)m0 * kMetaBytes;
-        bulk_to_peer(map_rank(su32(cbuf + cb_off), q), cbuf + cb_off, (uint32_t)nr * Lay::K, bar);
-        bulk_to_peer(map_rank(su32(reinterpret_cast<uint8_t*>(meta) + mt_off), q),
-                     reinterpret_cast<uint8_t*>(meta) + mt_off, (uint32_t)nr * kMetaBytes, bar);
+      // lane 0 of warp w sends to peers w, w + 8 (all peers but this CTA)
+      if (lane == 0 && nr > 0) {
+        for (uint32_t q = (uint32_t)warp; q < csize; q += kConsumers) {
+          if (q == crank) continue;
+          const uint32_t bar = map_rank(su32(codes_full), q);
+          const uint32_t cb_off = (uint32_t)m0 * Lay::K, mt_off = (uint32_t)m0 * kMetaBytes;
+          bulk_to_peer(map_rank(su32(cbuf + cb_off), q), cbuf + cb_off, (uint32_t)nr * Lay::K, bar);
+          bulk_to_peer(map_rank(su32(reinterpret_cast<uint8_t*>(meta) + mt_off), q),
+                       reinterpret_cast<uint8_t*>(meta) + mt_off, (uint32_t)nr * kMetaBytes, bar);
+        }
       }
       // the peers' rows
       ok = __all_sync(0xffffffffu, mbar_wait(codes_full, 0u, abort)) != 0;

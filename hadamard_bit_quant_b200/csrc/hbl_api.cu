@@ -650,8 +650,19 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 // ---------------------------------------------------------------------------
 constexpr int kFusedNotApplicable = -1;
 
-// Cluster size of the fused decode kernel: each CTA transforms two token rows.
-int fused_cluster_size(int M) { return M <= 2 ? 1 : (M <= 4 ? 2 : (M <= 8 ? 4 : 8)); }
+// Cluster size of the fused decode kernel: each CTA transforms ceil(M / size)
+// token rows (at most two). Preferred: one row per CTA (cluster size = M
+// rounded up to a power of two, 16-CTA clusters being non-portable); the
+// fallback, where such clusters cannot be scheduled, halves the size.
+#ifndef HBL_FUSED_ONE_ROW_MAX
+#define HBL_FUSED_ONE_ROW_MAX 16
+#endif
+int fused_cluster_size(int M) {
+  int cs = 1;
+  while (cs < M) cs <<= 1;
+  if (cs > HBL_FUSED_ONE_ROW_MAX) cs = (cs + 1) / 2;
+  return cs;
+}
 
 template <int LOG_K, int TN>
 int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const float* gain, const float* alpha,
@@ -659,11 +670,9 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   auto* kern = fdec::fused_decode_kernel<LOG_K, TN>;
   const size_t smem = fdec::Layout<LOG_K, 8 * TN>::kBytes;
   ensure_smem_attr(kern, smem);
-  const int CS = fused_cluster_size(M);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -673,30 +682,38 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = kUsePdl ? 2 : 1;
-  // clusters that fit at once (cached per device, kernel and cluster size)
+  // clusters of CS CTAs that fit at once (cached per device, kernel and cluster size)
   struct Entry { int dev; const void* fn; int cs; int clusters; };
   static std::mutex mu;
   static std::vector<Entry> known;
   int dev = 0;
   cudaGetDevice(&dev);
-  int clusters = -1;
-  {
+  auto clusters_of = [&](int CS) {
     std::lock_guard<std::mutex> lk(mu);
     for (auto& e : known)
-      if (e.dev == dev && e.fn == (const void*)kern && e.cs == CS) clusters = e.clusters;
-    if (clusters < 0) {
-      cfg.gridDim = dim3((unsigned)(sm_count / CS * CS));
-      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
-        (void)cudaGetLastError();
-        clusters = 0;
-      }
-      known.push_back(Entry{dev, (const void*)kern, CS, clusters});
+      if (e.dev == dev && e.fn == (const void*)kern && e.cs == CS) return e.clusters;
+    // clusters above 8 CTAs are opt-in (once per device and kernel, before the first launch)
+    if (CS > 8) (void)cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    attr[0].val.clusterDim.x = (unsigned)CS;
+    cfg.gridDim = dim3((unsigned)(sm_count / CS * CS));
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      clusters = 0;
     }
-  }
-  int grid = clusters * CS;
-  if (grid > sm_count / CS * CS) grid = sm_count / CS * CS;
+    known.push_back(Entry{dev, (const void*)kern, CS, clusters});
+    return clusters;
+  };
   const int groups = N / fdec::kGroupRows;
-  if (grid < CS || groups > fdec::kMaxGroups * grid || CS * fdec::kRowBatch < M) return kFusedNotApplicable;
+  int CS = fused_cluster_size(M), grid = 0;
+  for (;; CS /= 2) {
+    if (CS * fdec::kRowBatch < M) return kFusedNotApplicable;   // at most two rows per CTA
+    grid = clusters_of(CS) * CS;
+    if (grid > sm_count / CS * CS) grid = sm_count / CS * CS;
+    if (grid >= CS && groups <= fdec::kMaxGroups * grid) break;
+    if (CS == 1) return kFusedNotApplicable;
+  }
+  attr[0].val.clusterDim.x = (unsigned)CS;
   cfg.gridDim = dim3((unsigned)grid);
   ProfScope ps("fused_decode", s);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, X, M, N, gain, alpha, flags, Y);
