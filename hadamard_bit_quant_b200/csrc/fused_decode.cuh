@@ -9,20 +9,23 @@
 // plus a chain of short dependent steps (transform, statistic, codes, MMA,
 // epilogue). Two kernels cost two grid boundaries and an L2 round trip of the
 // codes; this kernel keeps every intermediate on chip:
-//   * one CTA per SM, grouped into clusters of CS CTAs (CS = 1, 2, 4 or 8);
+//   * one CTA per SM, grouped into clusters of CS CTAs (CS = 1, 2, 4, 8 or
+//     16: the token count rounded up to a power of two, halved where such
+//     clusters cannot be scheduled);
 //   * a producer warp streams the weights of the CTA's 16-row groups through
 //     a TMA ring ([16 rows][64 B] boxes, one per 256-k block) from the first
 //     instruction on, before the kernel waits for
 //     the grid that produced X (programmatic dependent launch);
-//   * the 8 consumer warps of cluster rank r transform and quantise token rows
-//     2r and 2r + 1 (256 threads per row, E = K/256 values per thread,
-//     butterflies in registers, passes exchanged through padded shared
-//     memory) into this CTA's shared memory: codes row-contiguous, scale and
-//     per-warp code sums beside them. Lane 0 of warp q then sends both rows to
-//     cluster rank q (every rank but this one) with two bulk copies (shared memory to
-//     distributed shared memory, completing as transaction bytes on the
-//     peer's mbarrier). Each CTA waits on its own barrier for the M - 2 rows
-//     it receives, so it holds all M x K codes;
+//   * the 8 consumer warps of cluster rank r transform and quantise token
+//     rows r*R .. r*R + R - 1, R = ceil(M / CS) <= 2 (256 threads per row,
+//     E = K/256 values per thread, butterflies in registers, passes exchanged
+//     through padded shared memory) into this CTA's shared memory: codes
+//     row-contiguous, scale and per-warp code sums beside them. Lane 0 of
+//     warp q then sends the rows to cluster ranks q and q + 8 (every rank but
+//     this one) with bulk copies (shared memory to distributed shared memory,
+//     completing as transaction bytes on the peer's mbarrier). Each CTA waits
+//     on its own barrier for the M - R rows it receives, so it holds all
+//     M x K codes;
 //   * the consumers then run the m16n8k32 MMAs of their groups (weights as A,
 //     u = t + 1 unpacked in registers; codes as B), batches of groups
 //     interleaved for independent accumulator chains, add the 8 warps' partial
@@ -71,6 +74,16 @@ HBL_DEVINL bool mbar_try_wait(uint64_t* b, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking probe (test_wait never suspends the thread).
+HBL_DEVINL bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
       : "r"(su32(b)), "r"(parity)
       : "memory");
@@ -397,11 +410,19 @@ HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, u
       }
     }
     uint32_t A4[NG][4], B4[NG][4];
+    // the NG unit barriers are probed back to back (their round trips overlap);
+    // only a unit still in flight is waited for
+    bool landed[NG];
+#pragma unroll
+    for (int b = 0; b < NG; ++b) {
+      const int u = c * NG + b;
+      landed[b] = mbar_test(&wfull[u % kStages], (uint32_t)(u / kStages) & 1u);
+    }
 #pragma unroll
     for (int b = 0; b < NG; ++b) {
       const int u = c * NG + b;
       const int s = u % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
+      if (!__all_sync(0xffffffffu, landed[b] || mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
       // block `warp` of the unit: box `warp`, [16 rows][64 B]; rows sit 64 B
       // apart, so the two rows a quarter-warp reads fall in different bank halves
       const uint8_t* wb = ring + (size_t)s * kUnitBytes + warp * (kGroupRows * 64);
