@@ -381,7 +381,9 @@ HBL_DEVINL void rows_phase(const uint16_t* __restrict__ X, int m0, bool had, boo
 // with one token tile, even and odd q accumulate separately). Codes are read
 // from the resident row-major buffer. Ends by writing this warp's partial sums
 // into shared memory (aliasing the ring) once every consumer is past its last
-// unit: red[warp][group][row][token].
+// unit: red[warp][group][token][row] (the epilogue's threads take consecutive
+// rows of one token, so its reads are free of bank conflicts and its stores
+// contiguous).
 template <int NG, int TN, int K>
 HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, uint64_t* wempty, volatile int* abort,
                           int warp, int lane) {
@@ -466,7 +468,7 @@ HBL_DEVINL bool fused_mma(uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, u
         for (int r = 0; r < 4; ++r) {
           const int row = g + ((r >> 1) << 3);
           const int tok = 8 * i + 2 * tig + (r & 1);
-          red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
+          red[((warp * kMaxGroups + gl) * MT + tok) * kGroupRows + row] = acc[gl][i][r];
         }
   }
   return ok;
@@ -617,7 +619,7 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
         if (tok < M) {
           int s = 0;
 #pragma unroll
-          for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * kGroupRows + row) * MT + tok];
+          for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * MT + tok) * kGroupRows + row];
           const uint32_t* mrow = meta + tok * (kMetaBytes / 4);
           int cs = 0;
 #pragma unroll

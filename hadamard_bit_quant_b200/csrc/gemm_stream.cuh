@@ -203,7 +203,9 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
       for (int r = 0; r < 4; ++r) acc[a][0][r] += acc[a][1][r];
   }
   // partial sums of the 8 warps -> shared memory (aliases the ring, so only
-  // after every warp is done with it): red[warp][group][row][token]
+  // after every warp is done with it): red[warp][group][token][row], so the
+  // epilogue's threads (consecutive rows of one token) read without bank
+  // conflicts
   asm volatile("bar.sync 1, %0;\n" ::"n"(kConsumers * 32) : "memory");
   if (ok && *abort == 0) {
     int* red = reinterpret_cast<int*>(ring);
@@ -215,7 +217,7 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
         for (int r = 0; r < 4; ++r) {
           const int row = g + ((r >> 1) << 3);
           const int tok = 8 * i + 2 * tig + (r & 1);
-          red[((warp * kMaxGroups + gl) * kGroupRows + row) * MT + tok] = acc[gl][i][r];
+          red[((warp * kMaxGroups + gl) * MT + tok) * kGroupRows + row] = acc[gl][i][r];
         }
   }
   return ok;
@@ -345,7 +347,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __re
       if (tok < M) {
         int s = 0;
 #pragma unroll
-        for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * kGroupRows + row) * MT + tok];
+        for (int w = 0; w < kConsumers; ++w) s += red[((w * kMaxGroups + gl) * MT + tok) * kGroupRows + row];
         s -= __ldg(csum + tok);
         if constexpr (OUT_BF16) {
           const float y = __fmul_rn(__fmul_rn((float)s, __ldg(scales + tok)), a);
