@@ -650,17 +650,16 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 // ---------------------------------------------------------------------------
 constexpr int kFusedNotApplicable = -1;
 
-// Cluster size of the fused decode kernel: each CTA transforms ceil(M / size)
-// token rows (at most two). Preferred: one row per CTA (cluster size = M
-// rounded up to a power of two, 16-CTA clusters being non-portable); the
-// fallback, where such clusters cannot be scheduled, halves the size.
-#ifndef HBL_FUSED_ONE_ROW_MAX
-#define HBL_FUSED_ONE_ROW_MAX 16
-#endif
+// Preferred cluster size of the fused decode kernel: one token row per CTA,
+// i.e. M rounded up to a power of two (16-CTA clusters are non-portable and
+// opted into at launch). Measured on B200 against two rows per CTA in half as
+// many CTAs, it is faster at every token count (M=16: 9.9 -> 9.2 us). Where
+// clusters of that size cannot be scheduled, or hold too few CTAs for the
+// row groups, launch_fused halves it (each CTA then transforms ceil(M / size)
+// rows, at most two).
 int fused_cluster_size(int M) {
   int cs = 1;
   while (cs < M) cs <<= 1;
-  if (cs > HBL_FUSED_ONE_ROW_MAX) cs = (cs + 1) / 2;
   return cs;
 }
 
