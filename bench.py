@@ -560,6 +560,31 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def profile_next(torch, hbl):
+    """The next rows' kernels, each called twice, at the sizes bench.py times them."""
+    g = torch.Generator().manual_seed(7)
+    M, K = 4096, 16384
+    X = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    gain = (0.5 + torch.rand(K, generator=g)).cuda()
+    codes = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    sc = torch.empty(M, device="cuda")
+    cs = torch.empty(M, dtype=torch.int32, device="cuda")
+    dXr = torch.randn(M, K, generator=g).cuda()
+    dX = torch.empty_like(dXr)
+    T, H, d = 4096, 32, 128
+    Xq = torch.randn(T, H, d, generator=g).to(torch.bfloat16).cuda()
+    cq = torch.empty(T, H, d, dtype=torch.uint8, device="cuda")
+    gq = torch.empty(T, H, device="cuda")
+    for _ in range(2):
+        hbl.hbl_quantize_ln(X, M, K, gain, 4, 1, codes, sc, cs)      # f1
+        hbl.hbl_hadamard_backward_f32(dXr, M, K, dX)                 # f3
+        hbl.hbl_quantize_qkv(Xq, T, H, d, 4, 0, cq, gq)              # f4
+    torch.cuda.synchronize()
+    assert hbl.hbl_get_device_error() == 0
+    print("profile case next: f1, f3, f4 kernels twice each ok")
+    return 0
+
+
 def profile_case(which: str):
     """A short, fixed run for ncu captures: pack once, then two forwards of one config."""
     import torch
@@ -572,6 +597,8 @@ def profile_case(which: str):
         case = [c for c in inputs.decode_oproj_cases((HEAD["M"],), (HEAD["act_bits"],))][0]
     elif which == "decode_big":
         case = inputs.sweep_case(16, 16384, 16384, 4, 1)
+    elif which == "next":
+        return profile_next(torch, hbl)
     else:
         raise SystemExit(f"unknown profile case {which}")
     X = case.make_x().cuda()
@@ -593,7 +620,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile-case", choices=["prefill", "decode", "decode_big"], default=None,
+    ap.add_argument("--profile-case", choices=["prefill", "decode", "decode_big", "next"], default=None,
                     help="run one short fixed case (for ncu captures) and exit")
     args = ap.parse_args()
     if args.profile_case:
