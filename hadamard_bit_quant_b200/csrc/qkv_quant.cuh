@@ -41,10 +41,16 @@ HBL_DEVINL void qkv_load(const uint16_t* src, float (&v)[VPL]) {
 }
 
 // Each warp quantises kQkvRowsPerWarp head vectors: their loads are all in
-// flight before the first reduction (the kernel is bound by HBM latency x
-// bytes in flight). x / (gamma + eps) is computed as x * (1 / (gamma + eps)),
-// one reciprocal per head; that moves q by at most an ulp, so a code can
-// differ from the exact division only at a rounding tie.
+// flight before the first reduction. Per head: gamma by one warp max
+// reduction over the bit patterns of |x| (for non-negative floats the bit
+// pattern orders like the value); r = 1 / (gamma + eps) correctly rounded
+// (the same value as the division); then per value
+//   q = x * (half_top * r) + half_top      (one fused multiply-add),
+// rounded to the nearest integer, ties to even, by adding 1.5 * 2^23 (the
+// integer then sits in the low bits), and packed four to a word. In exact
+// arithmetic q lies in [0, 2^b - 1] (|x| <= gamma < gamma + eps), and the
+// fp32 rounding moves it by far less than a half, so no clamp is needed; the
+// result can differ from the exact map only at a rounding tie.
 template <int VPL>
 __global__ void __launch_bounds__(256) qkv_quant_kernel(const uint16_t* __restrict__ X, int rows, int heads,
                                                         int bits, int bos_token, uint8_t* __restrict__ codes,
@@ -62,36 +68,49 @@ __global__ void __launch_bounds__(256) qkv_quant_kernel(const uint16_t* __restri
       for (int i = 0; i < VPL; ++i) v[r][i] = 0.f;
     }
   }
-  float g[R];
+  uint32_t gbits[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    g[r] = 0.f;
+    float m = 0.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) g[r] = fmaxf(g[r], fabsf(v[r][i]));
+    for (int i = 0; i < VPL; ++i) m = fmaxf(m, fabsf(v[r][i]));
+    gbits[r] = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-    for (int r = 0; r < R; ++r) g[r] = fmaxf(g[r], __shfl_xor_sync(0xffffffffu, g[r], off));
+  // rows [bos_lo, bos_hi) are the BOS token's heads
+  const long long bos_lo = bos_token >= 0 ? (long long)bos_token * heads : -1;
+  const long long bos_hi = bos_token >= 0 ? bos_lo + heads : -1;
+  const float2 magic = make_float2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int row = row0 + r;
     if (row >= rows) break;
-    const int b = (bos_token >= 0 && row / heads == bos_token) ? 8 : bits;
-    const int top = (1 << b) - 1;
-    const float half_top = 0.5f * (float)top;
-    const float rden = __fdiv_rn(1.f, __fadd_rn(g[r], kEps));
-    uint32_t packed[(VPL + 3) / 4] = {};
+    const float g = __uint_as_float(gbits[r]);
+    const int b = (row >= bos_lo && row < bos_hi) ? 8 : bits;
+    const float half_top = 0.5f * (float)((1 << b) - 1);
+    const float a = __fmul_rn(half_top, __frcp_rn(__fadd_rn(g, kEps)));
+    const float2 a2 = make_float2(a, a), h2 = make_float2(half_top, half_top);
+    uint32_t q[VPL];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const float x = __fmul_rn(half_top, __fadd_rn(__fmul_rn(v[r][i], rden), 1.f));
-      packed[i / 4] |= (uint32_t)clampi(__float2int_rn(x), 0, top) << (8 * (i % 4));
+    for (int i = 0; i < VPL; i += 2) {
+      const float2 t = __fadd2_rn(__ffma2_rn(make_float2(v[r][i], v[r][i + 1]), a2, h2), magic);
+      q[i] = __float_as_uint(t.x);
+      q[i + 1] = __float_as_uint(t.y);
+    }
+    // the low byte of each q is its code: bytes 0 of q0, q1 (, q2, q3) side by side
+    uint32_t packed[(VPL + 3) / 4];
+    if constexpr (VPL >= 4) {
+#pragma unroll
+      for (int w = 0; w < VPL / 4; ++w)
+        packed[w] = __byte_perm(__byte_perm(q[4 * w], q[4 * w + 1], 0x0040),
+                                __byte_perm(q[4 * w + 2], q[4 * w + 3], 0x0040), 0x5410);
+    } else {
+      packed[0] = __byte_perm(q[0], q[1], 0x0040) & 0xffffu;
     }
     uint8_t* dst = codes + (size_t)row * D + VPL * lane;
     if constexpr (VPL == 2) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed[0];
     else if constexpr (VPL == 4) *reinterpret_cast<uint32_t*>(dst) = packed[0];
     else *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    if (lane == 0) gamma_out[row] = g[r];
+    if (lane == 0) gamma_out[row] = g;
   }
 }
 
