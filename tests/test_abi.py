@@ -60,6 +60,19 @@ def test_host_side_queries(lib):
     assert hbl.hbl_workspace_bytes(0, 4096, 4096) >= 0
 
 
+def test_gemm_path_selector_bounds(lib):
+    # host-side only: the selector is a library global, checked before it is stored
+    from hadamard_bit_quant_b200 import hbl
+    raw = hbl.lib()
+    try:
+        for p in range(7):
+            assert raw.hbl_set_gemm_path(p) == 0
+        assert raw.hbl_set_gemm_path(-1) == 1
+        assert raw.hbl_set_gemm_path(7) == 1
+    finally:
+        assert raw.hbl_set_gemm_path(0) == 0
+
+
 BAD = 0x1000  # never dereferenced: every call below is rejected before any launch
 
 
