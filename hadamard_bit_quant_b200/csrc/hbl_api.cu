@@ -2,6 +2,7 @@
 // H-BitLinear forward (BitNet v2 architecture walkthrough, section 3.4, Eq. 9).
 // All kernels live in the headers included below (one translation unit, so the
 // device error word is shared).
+#include <atomic>
 #include <mutex>
 #include <cstring>
 #include <string>
@@ -410,8 +411,10 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 // 0 auto, 1 warp-level mma.sync, 2 tcgen05 persistent (128 x 128 tiles), 3 decode without
 // clusters or streaming, 4 tcgen05 one 128 x 256 tile per CTA (the default for M >= 128),
 // 5 weight-streaming decode (the default for M <= 16 where it fits), 6 as 0 (the forward
-// takes the fused single-kernel decode wherever it fits; 0 does the same)
-int g_gemm_path = 0;
+// takes the fused single-kernel decode wherever it fits; 0 does the same).
+// Every entry point reads it once and passes the value down, so one call never
+// mixes two settings.
+std::atomic<int> g_gemm_path{0};
 
 
 // Persistent tcgen05 kernel (one CTA per SM, 128 x 128 tiles, double-buffered accumulator).
@@ -487,8 +490,8 @@ enum class GemmKind { Decode, Mma, Tc, Tc2 };
 //    one 128 x 256 tile per CTA (half the weight re-reads of 128-token tiles);
 //  * otherwise the persistent tcgen05 kernel (128 x 128 tiles, accumulator
 //    double-buffered so the epilogue overlaps the next tile).
-GemmKind choose_gemm(int M, int K, int N) {
-  switch (g_gemm_path) {
+GemmKind choose_gemm(int M, int K, int N, int path) {
+  switch (path) {
     case 1: return GemmKind::Mma;
     case 2: return GemmKind::Tc2;
     case 4: return GemmKind::Tc;
@@ -614,15 +617,15 @@ int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 
 int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
                     const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s,
-                    int sm_count = 148) {
-  if ((g_gemm_path == 0 || g_gemm_path == 5 || g_gemm_path == 6) && stream_fits(M, K, N, sm_count)) {
+                    int sm_count, int path) {
+  if ((path == 0 || path == 5 || path == 6) && stream_fits(M, K, N, sm_count)) {
     const int st = run_gemm_stream(codes, M, K, N, Wpk, csum, scales, alpha, Y, acc, sm_count, s);
     if (st >= 0) return st;
   }
   {
     int C, KC;
     size_t sm;
-    if (g_gemm_path != 3 && decode2_config(M, K, &C, &KC, &sm))
+    if (path != 3 && decode2_config(M, K, &C, &KC, &sm))
       return run_gemm_decode2(codes, M, K, N, Wpk, csum, scales, alpha, Y, acc, s);
   }
   const int TN = M <= 8 ? 1 : (M <= 16 ? 2 : (M <= 32 ? 4 : 8));
@@ -760,16 +763,18 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   float* scales = reinterpret_cast<float*>(base + L.scales);
   int32_t* csum = reinterpret_cast<int32_t*>(base + L.csum);
   int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
-  if ((g_gemm_path == 0 || g_gemm_path == 6) && fused_fits(M, K, N)) {
+  const int path = g_gemm_path.load(std::memory_order_relaxed);
+  if ((path == 0 || path == 6) && fused_fits(M, K, N)) {
     const int fs = run_fused_decode(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, ln, gain, Y, d->sm_count, s);
     if (fs != kFusedNotApplicable) return fs;
   }
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
   if (st) return st;
-  switch (choose_gemm(M, K, N)) {
+  switch (choose_gemm(M, K, N, path)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
     case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
-    case GemmKind::Decode: return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count);
+    case GemmKind::Decode:
+      return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count, path);
     case GemmKind::Mma: break;
   }
   st = run_gemm(codes, M, K, N, Wpk, D, d->sm_count, s);
@@ -948,10 +953,12 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   }
   code_rowsum_kernel<<<M, 256, 0, s>>>(codes, K, csum);
   if ((st = launch_status())) return st;
-  switch (choose_gemm(M, K, N)) {
+  const int path = g_gemm_path.load(std::memory_order_relaxed);
+  switch (choose_gemm(M, K, N, path)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
     case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
-    case GemmKind::Decode: return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count);
+    case GemmKind::Decode:
+      return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count, path);
     case GemmKind::Mma: break;
   }
   if ((st = run_gemm(codes, M, K, N, Wpk, acc, d->sm_count, s))) return st;
@@ -1036,7 +1043,7 @@ int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_t
 
 int hbl_set_gemm_path(int path) {
   if (path < 0 || path > 6) return HBL_ERR_INVALID_ARG;
-  g_gemm_path = path;
+  g_gemm_path.store(path, std::memory_order_relaxed);
   return HBL_OK;
 }
 

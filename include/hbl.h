@@ -89,8 +89,12 @@ int hbl_pack_weights(const float* W, int N, int K, uint8_t* Wpk, float* wscale,
                      hbl_stream stream);
 
 /*
- * hbl_unpack_weights -- canonical view of packed weights.
- *   T : device int8, N x K row-major, written with codes in {-1, 0, +1}.
+ * hbl_unpack_weights -- canonical view of packed weights: the ternary codes
+ * RoundClip(W / (alpha + eps), -1, 1) of Eq. 1-2 (section 3.4, "Weight
+ * Quantization") that hbl_pack_weights stored.
+ *   Wpk : device, from hbl_pack_weights for an N x K matrix (same N, K).
+ *   T   : device int8, N x K row-major, written with codes in {-1, 0, +1}.
+ * Shapes as hbl_pack_weights. Asynchronous on `stream`; no allocation.
  */
 int hbl_unpack_weights(const uint8_t* Wpk, int N, int K, int8_t* T, hbl_stream stream);
 
@@ -169,17 +173,27 @@ int hbl_forward_noalloc(const hbl_bf16* X, int M, int K, int N, const uint8_t* W
 int hbl_hadamard_f32(const hbl_bf16* X, int M, int K, float* Xr, hbl_stream stream);
 
 /*
- * hbl_quantize -- optional Hadamard, then the per-token quantiser (Eq. 7 / Eq. 8).
+ * hbl_quantize -- optional Hadamard (Eq. 3-5), then the per-token quantiser
+ * (section 3.4, "Activation Quantization", Eq. 7 / Eq. 8).
  *   codes  : device int8 M x K.
  *   scales : device fp32 M: gamma/127 (act_bits 8) or beta/sqrt7 (act_bits 4).
- *   csum   : device int32 M or NULL: sum of the codes of each token.
+ *   csum   : device int32 M or NULL: sum of the codes of each token. Not part
+ *            of the method: the GEMM kernels multiply the codes by t + 1 (an
+ *            unsigned weight code) and subtract this sum, which is exact; it is
+ *            exposed so the stages can be checked one by one.
+ * Shapes as hbl_forward_ws (K a power of two in [256, 32768] with the
+ * Hadamard, else K % 256 == 0).
  */
 int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard,
                  int8_t* codes, float* scales, int32_t* csum, hbl_stream stream);
 
 /*
- * hbl_gemm_codes -- acc[m, n] = sum_k codes[m, k] * T[n, k], exactly, in int32.
+ * hbl_gemm_codes -- the integer product inside Eq. 9 (section 3.4,
+ * "H-BitLinear: The Composite Layer"), before any dequantisation:
+ * acc[m, n] = sum_k codes[m, k] * T[n, k], exactly, in int32, with T the
+ * ternary codes of Eq. 1-2 held in Wpk.
  *   codes : device int8 M x K (any values in [-128, 127]).
+ *   Wpk   : device, from hbl_pack_weights for an N x K matrix.
  *   acc   : device int32 M x N.
  * Same shape rules as hbl_forward_ws (K % 256 == 0). The per-token code
  * sums go to a small library-owned scratch that grows on demand (a
@@ -273,7 +287,10 @@ int hbl_get_device_error(hbl_stream stream);
  * forward, 6 = as 0.
  * All give results within the parity bounds of the oracle (the fused forward
  * and the quantiser kernel share their summation order, so the paths give the
- * same bits); the knob exists to check and time each one. Process-wide.
+ * same bits); the knob exists to check and time each one. Process-wide; each
+ * forward or hbl_gemm_codes call reads it once when it starts, so a change
+ * made while calls run on other threads applies from their next call on.
+ * Returns HBL_ERR_INVALID_ARG for a value outside 0..6.
  */
 int hbl_set_gemm_path(int path);
 

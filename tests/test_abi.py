@@ -98,11 +98,15 @@ def test_forward_argument_checks(lib, args, status):
     assert st == status
     st = lib.hbl_forward_ws(*args, BAD, 1 << 20, None)
     assert st == status
+    st = lib.hbl_forward_noalloc(*args, None)
+    assert st == status
 
 
 def test_empty_batch_is_a_noop(lib):
     # M == 0: nothing to do, nothing launched, HBL_OK even with null buffers
     assert lib.hbl_forward(None, 0, 4096, 4096, None, None, 4, 1, None, None) == 0
+    assert lib.hbl_forward_noalloc(None, 0, 4096, 4096, None, None, 4, 1, None, None) == 0
+    assert lib.hbl_forward_ws(None, 0, 4096, 4096, None, None, 4, 1, None, None, 0, None) == 0
     assert lib.hbl_quantize(None, 0, 4096, 4, 1, None, None, None, None) == 0
     assert lib.hbl_gemm_codes(None, 0, 4096, 4096, None, None, None) == 0
 
@@ -120,3 +124,14 @@ def test_quantize_and_hadamard_argument_checks(lib):
     assert lib.hbl_quantize(BAD, 2, 3000, 4, 1, BAD, BAD, None, None) == 2
     assert lib.hbl_hadamard_f32(BAD, 2, 3000, BAD, None) == 2
     assert lib.hbl_hadamard_f32(None, 2, 4096, BAD, None) == 1
+
+
+def test_noalloc_rejects_sizes_beyond_its_array(lib):
+    # the fixed 8 MiB array: a size whose workspace exceeds it is refused before
+    # any device work (HBL_ERR_WORKSPACE), one that fits passes the size check
+    from hadamard_bit_quant_b200 import hbl
+    assert hbl.hbl_workspace_bytes(4096, 16384, 256) > 8 << 20
+    assert lib.hbl_forward_noalloc(BAD, 4096, 16384, 256, BAD, BAD, 4, 1, BAD, None) == 7
+    assert hbl.hbl_workspace_bytes(16, 4096, 4096) <= 8 << 20
+    # still refused on its arguments first
+    assert lib.hbl_forward_noalloc(BAD, 4096, 16384, 256, BAD, BAD, 5, 1, BAD, None) == 1

@@ -69,6 +69,34 @@ def test_hadamard_f32(L, K):
     parity.check_hadamard(Xr, ref)
 
 
+# Batches above the few-token threshold (64 tokens) take the throughput
+# configurations of the transform (more values per thread, several tokens per
+# CTA for small K); each K is checked there too, with ragged CTA tails, on
+# sampled tokens (tokens are independent, so a sampled row is exact).
+@pytest.mark.parametrize("K,M", [(256, 65), (512, 70), (1024, 129), (2048, 100), (4096, 257), (8192, 97),
+                                 (16384, 130), (32768, 66)])
+def test_hadamard_f32_many_tokens(L, K, M):
+    X = inputs.gaussian_with_outliers(M, K, 20 + K, inputs.outlier_channels(K, 0.01, 3).tolist(), 50.0)
+    rng = np.random.default_rng(K)
+    rows = np.unique(np.concatenate([[0, 1, M - 2, M - 1], rng.integers(0, M, 12)]))
+    Xr = L.hadamard_f32(dev(X)).cpu().numpy()[rows]
+    ref = oracle.hadamard(X[rows].to(torch.float64).numpy())
+    parity.check_hadamard(Xr, ref)
+
+
+def test_hadamard_f32_prefill_shape(L):
+    """The prefill down_proj input (M=4096, K=16384, gated heavy-tailed values):
+    the transform's fp32 output on 40 sampled tokens, first and last included."""
+    case = inputs.prefill_down_case()
+    X = case.make_x()
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([[0, 1, 4094, 4095], rng.integers(0, case.M, 36)]))
+    Xr = L.hadamard_f32(dev(X)).cpu().numpy()[rows]
+    ref = oracle.hadamard(X[rows].to(torch.float64).numpy())
+    assert len(rows) >= 32
+    parity.check_hadamard(Xr, ref)
+
+
 def test_hadamard_special_rows(L):
     K = 4096
     X = torch.zeros(4, K)

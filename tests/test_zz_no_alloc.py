@@ -6,13 +6,13 @@ serving process whose pool already holds nearly all of HBM, code that cannot
 afford the synchronisation of cudaMalloc/cudaFree, hosts that forbid plugin
 allocations). Its workspace is a fixed device array shared by every call, so
 the test runs each case twice in a row: the second call must not see stale
-state from the first. This file is collected last on purpose.
+state from the first. Both entry points run the same kernels on the same
+inputs, so their outputs must be identical bit for bit. This file is
+collected last on purpose.
 """
-import numpy as np
 import pytest
 import torch
 
-import parity
 from hadamard_bit_quant_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -28,29 +28,48 @@ def H():
 
 
 CASES = [
-    # M, K, N, act_bits, use_hadamard
-    (16, 4096, 4096, 4, 1),    # decode-shaped o_proj, W1.58A4
-    (3, 1024, 256, 8, 0),      # plain BitLinear, INT8
-    (100, 4096, 512, 4, 1),    # warp-level GEMM path: split-K partials accumulate in the workspace
+    # M, K, N, act_bits, use_hadamard, GEMM path (0 = by size, 1 = warp-level split-K)
+    (16, 4096, 4096, 4, 1, 0),     # decode-shaped o_proj, W1.58A4 (fused kernel: no workspace use)
+    (3, 1024, 256, 8, 0, 0),       # plain BitLinear, INT8
+    (100, 4096, 512, 4, 1, 1),     # split-K: codes, scales and int32 partials all live in the workspace
+    (200, 2048, 1024, 8, 1, 2),    # persistent tcgen05 GEMM reading codes from the workspace
 ]
 
 
-@pytest.mark.parametrize("M,K,N,a,h", CASES)
-def test_noalloc_matches_workspace_forward(H, M, K, N, a, h):
+def _kernels_of(H, fn):
+    """Names of the library kernels one call launches (the library's own launch profile)."""
+    H.hbl_profile_enable(1)
+    fn()
+    torch.cuda.synchronize()
+    names = set(H.profile_table())
+    H.hbl_profile_enable(0)
+    return names
+
+
+@pytest.mark.parametrize("M,K,N,a,h,path", CASES)
+def test_noalloc_matches_workspace_forward(H, M, K, N, a, h, path):
     from hadamard_bit_quant_b200 import layer
     X = inputs.student_t(M, K, 11 + M).cuda()
     Wpk, wsc = layer.pack_weights(inputs.gaussian_weights(N, K, 12 + N).cuda())
     ws = layer.workspace(M, K, N, "cuda")
     ref = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-    H.hbl_forward_ws(X, M, K, N, Wpk, wsc, a, h, ref, ws, ws.numel())
-    yref = ref.float().cpu().numpy()
-    for call in range(2):
-        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-        H.hbl_forward_noalloc(X, M, K, N, Wpk, wsc, a, h, Y)
-        torch.cuda.synchronize()
-        y = Y.float().cpu().numpy()
-        assert np.all(np.isfinite(y)), f"call {call}: output not fully written"
-        assert np.all(np.abs(y - yref) <= parity.Y_RTOL * np.abs(yref)), f"call {call}"
+    H.hbl_set_gemm_path(path)
+    try:
+        H.hbl_forward_ws(X, M, K, N, Wpk, wsc, a, h, ref, ws, ws.numel())
+        # dirty the shared array with another size first, so stale contents would show
+        Xo = inputs.student_t(37, 1024, 5).cuda()
+        Wo, ao = layer.pack_weights(inputs.gaussian_weights(64, 1024, 6).cuda())
+        H.hbl_forward_noalloc(Xo, 37, 1024, 64, Wo, ao, 4, 1,
+                              torch.empty(37, 64, dtype=torch.bfloat16, device="cuda"))
+        for call in range(2):
+            Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+            names = _kernels_of(H, lambda: H.hbl_forward_noalloc(X, M, K, N, Wpk, wsc, a, h, Y))
+            if path == 1:
+                # the path that zeroes and accumulates into the shared array really ran
+                assert {"memset_acc", "gemm_mma"} <= names, names
+            assert torch.equal(Y, ref), f"call {call}: differs from hbl_forward_ws"
+    finally:
+        H.hbl_set_gemm_path(0)
     assert H.hbl_get_device_error() == 0
 
 
