@@ -143,6 +143,71 @@ class ClockSampler:
                 "power_w_max": max(r["power"] for r in rows)}
 
 
+class ClockPoller:
+    """SM clock and clock-event (throttle) reasons read through NVML from a background
+    thread every ~0.5 ms while running: read-only queries, fine-grained enough for a timed
+    region of a few milliseconds (nvidia-smi samples every 200 ms at best)."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch, local, period_s=0.0005):
+        self.torch, self.local, self.period = torch, local, period_s
+        self.samples, self.thread, self.h, self.nv = [], None, None, None
+        self.stop_flag = False
+
+    def _handle(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        self.nv = nv
+        try:
+            uuid = str(self.torch.cuda.get_device_properties(self.local).uuid)
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(gpu_index(self.torch, self.local))
+
+    def _reasons(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return f(self.h)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        import threading
+        try:
+            self.h = self._handle()
+            self.smax = self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_flag = True
+        self.thread.join(2)
+        if not self.samples:
+            return None
+        reasons = set()
+        for _, r in self.samples:
+            for bit, nm in self.REASONS.items():
+                if r & bit:
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": float(self.smax),
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "sm_mhz_min": min(c for c, _ in self.samples),
+                "source": "NVML clock and clock-event reasons polled every 0.5 ms during the timed region"}
+
+
 # ----------------------------------------------------------------------------- workloads
 def headline_workload_name():
     return (f"prefill_down M={HEAD['M']} K={HEAD['K']} N={HEAD['N']} W1.58A{HEAD['act_bits']} "
@@ -344,8 +409,8 @@ def prefill_headline(torch, dist, hbl, layer, inputs, args, world, local, peaks,
 
     fwd(0)
     torch.cuda.synchronize()
-    clocks = ClockSampler(gpu_index(torch, local))
-    clocks.start()
+    smi = ClockSampler(gpu_index(torch, local))
+    smi.start()
     for i in range(args.warmup):
         fwd(i)
     torch.cuda.synchronize()
@@ -355,15 +420,20 @@ def prefill_headline(torch, dist, hbl, layer, inputs, args, world, local, peaks,
     hbl.hbl_profile_enable(1)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    poll = ClockPoller(torch, local)
+    poll.start()
     e0.record()
     for i in range(args.steps):
         fwd(i)
     e1.record()
     torch.cuda.synchronize()
+    clk = poll.stop()
     ms = e0.elapsed_time(e1)
     prof = prof_dict(hbl)
     hbl.hbl_profile_enable(0)
-    clk = clocks.stop()
+    clk_smi = smi.stop()
+    if clk is None:
+        clk = clk_smi
     if world > 1:
         from hadamard_bit_quant_b200.shard import max_over_ranks
         ms = max_over_ranks(ms, device="cuda")
@@ -441,7 +511,8 @@ def prefill_headline(torch, dist, hbl, layer, inputs, args, world, local, peaks,
            "copies": "per step, pinned host <-> device on two copy streams beside the compute stream"}
     gpu_launches = sum(v["launches"] for k, v in prof.items() if k != "memset_acc")
     out = {"value": tokens / (ms * 1e-3), "ms": ms, "tops": ops * world * args.steps / (ms * 1e-3) / 1e12,
-           "roofline": roof, "kernels": kt, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clk}
+           "roofline": roof, "kernels": kt, "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clk,
+           "clocks_smi": clk_smi}
     del X, W, Y, ws, Xd, Yd
     torch.cuda.empty_cache()
     return out
@@ -749,6 +820,7 @@ def run_ours(args, rank, world, local):
         "e2e": head["e2e"],
         "gpu_launches": head["gpu_launches"],
         "clocks": head["clocks"],
+        "clocks_smi_whole_warmup_and_timed": head["clocks_smi"],
     }
     if rank == 0 and world == 1 and not args.no_extras:
         for key, fn in (("decode", lambda: decode_roofline(torch, hbl, layer, inputs, peaks, peak_kind)),
