@@ -127,7 +127,7 @@ HBL_DEVINL void convert_row(const uint8_t* tile, int row, uint32_t taddr) {
 }
 
 template <bool OUT_BF16>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_tcw_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_w, int M,
                 int K, int N, const int32_t* __restrict__ csum, const float* __restrict__ scales,
                 const float* __restrict__ alpha, uint16_t* __restrict__ Y, int32_t* __restrict__ acc_out) {
