@@ -5,19 +5,22 @@
 // Layer", Eq. 9: acc[m, n] = sum_k c[m, k] * t[n, k], then the dequant
 // acc * s[m] * alpha (Eq. 1, Eq. 7 / Eq. 8).
 //
-// One CTA computes a 128 (output features) x TOKS (tokens: 128, 192 or 256) tile of D = sum c*u
-// (u = t + 1 in {0,1,2}; the exact product is D - sum_k c):
+// One CTA computes a 128 (output features) x 256 (tokens) tile of D = sum c*u
+// (u = t + 1 in {0,1,2}; the exact product is D - sum_k c). When the tiles do
+// not fill the last wave of CTAs (one CTA per SM), the tiles of that wave are
+// split into two 128-token halves run by two CTAs, so the wave takes about half
+// as long (the tail CTAs carry the highest indices and start last):
 //   * warp 0 (one lane): TMA producer. Per 256-k stage it loads the codes
-//     tile (TOKS tokens x 256 k, two 128-byte-wide boxes, 128B swizzle) and the
-//     packed weight tile (128 rows x 64 bytes, 64B swizzle).
+//     tile (256 or 128 tokens x 256 k, two 128-byte-wide boxes, 128B swizzle)
+//     and the packed weight tile (128 rows x 64 bytes, 64B swizzle).
 //   * warps 2..5: converters. Each thread owns one weight row (one TMEM lane),
 //     unpacks its 64 packed bytes into 256 unsigned bytes in registers and
 //     writes them into the stage's 64 TMEM columns with tcgen05.st. The
 //     weights thus become the MMA's A operand straight from tensor memory and
 //     never pass through shared memory unpacked.
 //   * warp 1 (one lane): MMA issuer. Eight tcgen05.mma.kind::i8 (M=128,
-//     N=TOKS, K=32) per stage, A from TMEM, B (codes) from shared memory,
-//     int32 accumulator in TMEM columns [0, TOKS); tcgen05.commit frees the stage.
+//     N=256 or 128, K=32) per stage, A from TMEM, B (codes) from shared memory,
+//     int32 accumulator in TMEM columns [0, N); tcgen05.commit frees the stage.
 //   * warps 2..5 again: epilogue. tcgen05.ld of the accumulator, subtract the
 //     code sum, scale by s[m] * alpha, store bf16 (or the int32 result).
 // Every mbarrier wait is bounded (about a second of clock cycles); on timeout
@@ -38,30 +41,43 @@ constexpr int kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr long long kSpinLimit = 4000000000ll;    // ~2 s of SM clock
 
-// TOKS tokens per tile (the MMA's N, a multiple of 64 from 128 to 256; the
-// launcher uses 256).
-template <int TOKS>
-struct Tile {
-  static_assert(TOKS % 64 == 0 && TOKS >= 128 && TOKS <= 256, "token tile");
-  static constexpr int kBBytes = TOKS * kKBlock;          // codes per stage (two [TOKS][128 B] boxes)
-  static constexpr int kStageTx = kBBytes + kABytes;
-  static constexpr int kDCols = TOKS;                     // accumulator columns
-  static_assert(kDCols + kStages * kACols <= kTmemCols, "TMEM columns");
-  struct __align__(8) Smem {
-    uint8_t b[kStages][kBBytes];      // 1024-byte aligned (swizzle atoms)
-    uint8_t a[kStages][kABytes];
-    uint64_t full[kStages];
-    uint64_t aready[kStages];
-    uint64_t empty[kStages];
-    uint64_t done;
-    uint32_t tmem_base;
-    int abort;
-  };
-  static constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
-  // Instruction descriptor: D s32, A u8, B s8, both K-major, M = 128, N = TOKS.
-  static constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(TOKS >> 3) << 17) |
-                                     ((uint32_t)(kRows >> 4) << 24);
+constexpr int kToks = 256;                        // tokens of a full tile (MMA N)
+constexpr int kBBytes = kToks * kKBlock;          // codes per stage (two [256][128 B] boxes)
+constexpr int kDCols = kToks;                     // accumulator columns (A stages follow)
+static_assert(kDCols + kStages * kACols <= kTmemCols, "TMEM columns");
+
+struct __align__(8) Smem {
+  uint8_t b[kStages][kBBytes];      // 1024-byte aligned (swizzle atoms)
+  uint8_t a[kStages][kABytes];
+  uint64_t full[kStages];
+  uint64_t aready[kStages];
+  uint64_t empty[kStages];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
 };
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+
+// Instruction descriptor: D s32, A u8, B s8, both K-major, M = 128, N = toks.
+HBL_DEVINL uint32_t idesc_for(int toks) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(toks >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+}
+
+// Tile of CTA b: CTAs [0, full) own 128 x 256 tiles (output rows fastest);
+// each later pair of CTAs splits one of the remaining tiles into two
+// 128-token halves.
+HBL_DEVINL void cta_tile(int b, int full, int n_tiles, int* n0, int* m0, int* toks) {
+  if (b < full) {
+    *n0 = (b % n_tiles) * kRows;
+    *m0 = (b / n_tiles) * kToks;
+    *toks = kToks;
+  } else {
+    const int h = b - full, t = full + h / 2;
+    *n0 = (t % n_tiles) * kRows;
+    *m0 = (t / n_tiles) * kToks + (h & 1) * (kToks / 2);
+    *toks = kToks / 2;
+  }
+}
 
 HBL_DEVINL uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -168,20 +184,20 @@ HBL_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
       : "memory")
 
 // OUT_BF16: Y = bf16((D - csum) * s * alpha); else acc (int32) = D - csum.
-template <bool OUT_BF16, int TOKS>
+// map_codes loads 256-token boxes, map_codes_half 128-token boxes (split tiles).
+template <bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_w, int M,
-               int K, int N, const int32_t* __restrict__ csum, const float* __restrict__ scales,
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_codes_half,
+               const __grid_constant__ CUtensorMap map_w, int M, int K, int N, int full,
+               const int32_t* __restrict__ csum, const float* __restrict__ scales,
                const float* __restrict__ alpha, uint16_t* __restrict__ Y, int32_t* __restrict__ acc_out) {
-  using TL = Tile<TOKS>;
-  using Smem = typename TL::Smem;
-  constexpr int kBBytes = TL::kBBytes, kStageTx = TL::kStageTx, kDCols = TL::kDCols;
-  constexpr uint32_t kIdesc = TL::kIdesc;
   extern __shared__ uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kRows;
-  const int m0 = blockIdx.y * TOKS;
+  int n0, m0, toks;
+  cta_tile(blockIdx.x, full, (N + kRows - 1) / kRows, &n0, &m0, &toks);
+  const int bbytes = toks * kKBlock;                 // codes bytes per stage
+  const uint32_t idesc = idesc_for(toks);
   const int nblk = K / kKBlock;
   volatile int* abort = &S.abort;
 
@@ -214,9 +230,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
         const int s = kb % kStages;
         const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
         if (kb >= kStages && !mbar_wait(&S.empty[s], ph ^ 1u, abort)) break;
-        mbar_expect_tx(&S.full[s], kStageTx);
-        tma_load_2d(&S.b[s][0], &map_codes, &S.full[s], kb * kKBlock, m0);
-        tma_load_2d(&S.b[s][kBBytes / 2], &map_codes, &S.full[s], kb * kKBlock + 128, m0);
+        const CUtensorMap* mc = toks == kToks ? &map_codes : &map_codes_half;
+        mbar_expect_tx(&S.full[s], (uint32_t)(bbytes + kABytes));
+        tma_load_2d(&S.b[s][0], mc, &S.full[s], kb * kKBlock, m0);
+        tma_load_2d(&S.b[s][bbytes / 2], mc, &S.full[s], kb * kKBlock + 128, m0);
         tma_load_2d(&S.a[s][0], &map_w, &S.full[s], kb * (kKBlock / 4), n0);
         ++issued;
       }
@@ -241,8 +258,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
 #pragma unroll
         for (int j = 0; j < kKBlock / 32; ++j) {
           const uint32_t a_addr = tmem + (uint32_t)(kDCols + s * kACols + 8 * j);
-          const uint64_t bdesc = smem_desc_sw128(bbase + (uint32_t)((j >> 2) * (kBBytes / 2) + (j & 3) * 32));
-          mma_i8_ts(tmem, a_addr, bdesc, kIdesc, (kb > 0 || j > 0) ? 1u : 0u);
+          const uint64_t bdesc = smem_desc_sw128(bbase + (uint32_t)((j >> 2) * (bbytes / 2) + (j & 3) * 32));
+          mma_i8_ts(tmem, a_addr, bdesc, idesc, (kb > 0 || j > 0) ? 1u : 0u);
         }
         tc_commit(&S.empty[s]);
         ++issued;
@@ -295,7 +312,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
       const int n = n0 + row;
       const float a = OUT_BF16 ? __ldg(alpha) : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < kDCols / 32; ++c) {
+      for (int c = 0; c < toks / 32; ++c) {
         uint32_t d[32];
         HBL_TMEM_LD32(tmem + lane_addr + (uint32_t)(32 * c), d);
         tc_wait_ld();

@@ -442,38 +442,36 @@ int run_gemm_tc2(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, c
   return launch_status();
 }
 
-// bf16 output (Y != nullptr) or int32 output (acc != nullptr); D - csum either way.
-template <int TOKS>
-int launch_gemm_tc(const CUtensorMap& mc, const CUtensorMap& mw, int M, int K, int N, const int32_t* csum,
-                   const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, cudaStream_t s) {
-  using TL = tc::Tile<TOKS>;
-  const dim3 grid((N + tc::kRows - 1) / tc::kRows, (M + TOKS - 1) / TOKS);
-  ProfScope ps("gemm_tc", s);
-  if (Y) {
-    ensure_smem_attr(tc::gemm_tc_kernel<true, TOKS>, TL::kSmemBytes);
-    tc::gemm_tc_kernel<true, TOKS><<<grid, tc::kThreads, TL::kSmemBytes, s>>>(mc, mw, M, K, N, csum, scales, alpha,
-                                                                               Y, nullptr);
-  } else {
-    ensure_smem_attr(tc::gemm_tc_kernel<false, TOKS>, TL::kSmemBytes);
-    tc::gemm_tc_kernel<false, TOKS><<<grid, tc::kThreads, TL::kSmemBytes, s>>>(mc, mw, M, K, N, csum, nullptr,
-                                                                                nullptr, nullptr, acc);
-  }
-  return launch_status();
-}
-
-// One-tile-per-CTA tcgen05 GEMM with 128 x 256 tiles. (Measured on B200 over
-// prefill shapes, 256-token tiles beat 192 and 128 everywhere even where
-// narrower tiles fill the last wave better: the kernel is bound by feeding
-// codes from L2, and a wider tile re-reads the weights less.)
+// One-tile-per-CTA tcgen05 GEMM with 128 x 256 tiles (measured on B200 over
+// prefill shapes: 256-token tiles beat 192 and 128 as the tile of a full wave,
+// since a wider tile re-reads the weights less). When the tiles leave the last
+// wave of CTAs at most half full, that wave's tiles are split into 128-token
+// halves (twice the CTAs, each half as long), which shortens the wave instead
+// of leaving SMs idle. bf16 output (Y != nullptr) or int32 output (acc).
 int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
                 const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count, cudaStream_t s) {
-  (void)sm_count;
-  constexpr int toks = 256;
-  CUtensorMap mc, mw;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)toks, 128)) return HBL_ERR_CUDA;
+  CUtensorMap mc, mch, mw;
+  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)tc::kToks, 128))
+    return HBL_ERR_CUDA;
+  if (!make_map_u8(&mch, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, (uint32_t)tc::kToks / 2, 128))
+    return HBL_ERR_CUDA;
   if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tc::kRows, 64))
     return HBL_ERR_CUDA;
-  return launch_gemm_tc<toks>(mc, mw, M, K, N, csum, scales, alpha, Y, acc, s);
+  const int tiles = ((N + tc::kRows - 1) / tc::kRows) * ((M + tc::kToks - 1) / tc::kToks);
+  const int tail = sm_count > 0 ? tiles % sm_count : 0;
+  const int full = (tail > 0 && 2 * tail <= sm_count) ? tiles - tail : tiles;
+  const dim3 grid((unsigned)(full + 2 * (tiles - full)));
+  ProfScope ps("gemm_tc", s);
+  if (Y) {
+    ensure_smem_attr(tc::gemm_tc_kernel<true>, tc::kSmemBytes);
+    tc::gemm_tc_kernel<true><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(mc, mch, mw, M, K, N, full, csum, scales,
+                                                                         alpha, Y, nullptr);
+  } else {
+    ensure_smem_attr(tc::gemm_tc_kernel<false>, tc::kSmemBytes);
+    tc::gemm_tc_kernel<false><<<grid, tc::kThreads, tc::kSmemBytes, s>>>(mc, mch, mw, M, K, N, full, csum, nullptr,
+                                                                          nullptr, nullptr, acc);
+  }
+  return launch_status();
 }
 
 // Persistent tcgen05 kernel with 256 weight rows x 128 tokens per tile (each
