@@ -362,145 +362,6 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
   }
 }
 
-// Persistent form of the kernel above for configurations with one token per
-// CTA (T >= 128 threads), for many tokens: each CTA walks the tokens
-// blockIdx.x, blockIdx.x + gridDim.x, ... and fetches the next token's row by
-// one bulk copy while the current token is transformed, so the row's HBM
-// latency hides behind the butterflies instead of stalling every token.
-//   STAGED = true: the row lands in a staging buffer of its own (K * 2 or
-//     K * 4 bytes beside the exchange buffer); the next copy is issued as soon
-//     as the current row has been read into registers.
-//   STAGED = false: the row lands in the exchange buffer itself; the next
-//     copy is issued once the last pass has read its values from it (less
-//     shared memory, so more CTAs per SM, but a shorter overlap).
-// Same arithmetic, order of operations and results as fwht_quant_kernel.
-template <int LOG_K, int G, int MODE, bool IN_F32, bool LN, bool STAGED>
-__global__ void __launch_bounds__(FwhtCfg<LOG_K, G>::THREADS)
-fwht_quant_persist_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ gain,
-                          int8_t* __restrict__ codes, float* __restrict__ scales, int32_t* __restrict__ csum,
-                          float* __restrict__ Xr) {
-  using C = FwhtCfg<LOG_K, G>;
-  static_assert(C::TPC == 1, "one token per CTA");
-  constexpr int K = C::K, E = C::E, T = C::T, P = C::P;
-  extern __shared__ __align__(16) float smem[];
-  __shared__ float red_f[C::WARPS_PER_TOKEN];
-  __shared__ int red_i[C::WARPS_PER_TOKEN];
-  __shared__ __align__(8) uint64_t stage_bar;
-  float* sm = smem;                                               // exchange buffer
-  const void* stage = STAGED ? static_cast<const void*>(smem + C::KPAD) : static_cast<const void*>(smem);
-  const int t = threadIdx.x;
-  constexpr uint32_t kRowBytes = (uint32_t)K * (IN_F32 ? 4u : 2u);
-  const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&stage_bar);
-  const uint32_t stage_s = (uint32_t)__cvta_generic_to_shared(stage);
-
-  if (t == 0) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
-  __syncthreads();
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  // one thread fetches row r into the staging area (after ordering the CTA's
-  // earlier generic-proxy reads of that area before the asynchronous write)
-  auto fetch = [&](size_t r) {
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(kRowBytes) : "memory");
-    const char* src = reinterpret_cast<const char*>(Xv) + r * (size_t)kRowBytes;
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                     stage_s),
-                 "l"(src), "r"(kRowBytes), "r"(bar)
-                 : "memory");
-  };
-  size_t m = blockIdx.x;
-  if (t == 0 && m < (size_t)M) fetch(m);
-  for (uint32_t it = 0; m < (size_t)M; ++it, m += gridDim.x) {
-    const size_t next = m + gridDim.x;
-    {
-      uint32_t done = 0;
-      const long long t0 = clock64();
-      while (true) {
-        asm volatile(
-            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(done)
-            : "r"(bar), "r"(it & 1u)
-            : "memory");
-        if (done || clock64() - t0 > 4000000000ll) break;
-      }
-      if (!done) {   // give up on the rest of this CTA's tokens (the copy may still land: wait for it, bounded)
-        if (t == 0) set_device_error(HBL_ERR_TIMEOUT);
-        const long long t1 = clock64();
-        while (!done && clock64() - t1 < 4000000000ll) {
-          asm volatile(
-              "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-              : "=r"(done)
-              : "r"(bar), "r"(it & 1u)
-              : "memory");
-        }
-        break;
-      }
-    }
-    float v[E];
-    float ssq = 0.f;
-    // Pass 0 owns the top G bits: idx = t + j*T.
-    if constexpr (IN_F32) {
-      const float* row = static_cast<const float*>(stage);
-#pragma unroll
-      for (int j = 0; j < E; ++j) v[j] = row[t + j * T];
-    } else {
-      const uint16_t* row = static_cast<const uint16_t*>(stage);
-#pragma unroll
-      for (int j = 0; j < E; ++j) v[j] = bf16_bits_to_float(row[t + j * T]);
-    }
-    if constexpr (LN) {
-#pragma unroll
-      for (int j = 0; j < E; ++j) ssq = __fmaf_rn(v[j], v[j], ssq);
-      if (gain) {
-#pragma unroll
-        for (int j = 0; j < E; ++j) v[j] = __fmul_rn(v[j], __ldg(gain + t + j * T));
-      }
-    }
-    __syncthreads();   // the row is consumed: its buffer may be refilled / overwritten
-    if constexpr (STAGED) {
-      if (t == 0 && next < (size_t)M) fetch(next);
-    }
-#pragma unroll
-    for (int p = 0; p < P; ++p) {
-      const int hi = LOG_K - p * G;
-      const int lo = hi - G > 0 ? hi - G : 0;
-      const int nb = hi - lo;
-      if (p > 0) {
-        const int hi_prev = LOG_K - (p - 1) * G;
-        const int lo_prev = hi_prev - G > 0 ? hi_prev - G : 0;
-#pragma unroll
-        for (int j = 0; j < E; ++j) sm[pad<G, C::PADW>(pass_index<G>(t, j, lo_prev))] = v[j];
-        __syncthreads();
-        if (C::PADW == 4 && lo == 0) {
-          const float4* src = reinterpret_cast<const float4*>(sm + t * (E + 4));
-#pragma unroll
-          for (int q = 0; q < E / 4; ++q) {
-            const float4 f = src[q];
-            v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < E; ++j) v[j] = sm[pad<G, C::PADW>(pass_index<G>(t, j, lo))];
-        }
-        __syncthreads();
-        if constexpr (!STAGED) {
-          // the last pass has its values: the exchange buffer takes the next row
-          if (p + 1 == P && t == 0 && next < (size_t)M) fetch(next);
-        }
-      }
-      butterflies<E>(v, nb);
-    }
-    float nrm = __uint_as_float((uint32_t)(127 - LOG_K / 2) << 23);
-    if (LOG_K & 1) nrm *= 0.70710678118654752f;
-    if constexpr (LN) {
-      const float tot = token_reduce_f<T, C::WARPS_PER_TOKEN, false>(ssq, red_f, 0);
-      const float r = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, (float)K), kRmsEps)));
-      nrm = __fmul_rn(nrm, r);
-    }
-    quant_tail<E, T, C::WARPS_PER_TOKEN, MODE>(v, K, t, 0, true, m, red_f, red_i, codes, scales, csum, Xr, nrm);
-  }
-}
-
 // Plain per-token quantiser (no Hadamard), K % 256 == 0, one token per CTA,
 // thread t holds the E consecutive values [E*t, E*t + E).
 template <int E, int MODE, bool LN = false>

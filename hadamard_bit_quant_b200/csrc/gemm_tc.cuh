@@ -34,8 +34,7 @@ namespace hbl {
 namespace tc {
 
 constexpr int kRows = 128;         // weight rows per tile (MMA M)
-constexpr int kStages = 4;         // weight stages (256 k each), also the TMEM A stages
-constexpr int kCStages = 6;        // code stages (128 k each)
+constexpr int kStages = 3;
 constexpr int kABytes = kRows * (kKBlock / 4);    // 8 KB packed weights per stage
 constexpr int kACols = kKBlock / 4;               // 64 TMEM columns of A per stage
 constexpr int kTmemCols = 512;
@@ -43,18 +42,16 @@ constexpr int kThreads = 192;
 constexpr long long kSpinLimit = 4000000000ll;    // ~2 s of SM clock
 
 constexpr int kToks = 256;                        // tokens of a full tile (MMA N)
-constexpr int kCBytes = kToks * 128;              // codes per stage: one [256][128 B] box (128 k)
+constexpr int kBBytes = kToks * kKBlock;          // codes per stage (two [256][128 B] boxes)
 constexpr int kDCols = kToks;                     // accumulator columns (A stages follow)
 static_assert(kDCols + kStages * kACols <= kTmemCols, "TMEM columns");
 
 struct __align__(8) Smem {
-  uint8_t b[kCStages][kCBytes];     // 1024-byte aligned (swizzle atoms)
+  uint8_t b[kStages][kBBytes];      // 1024-byte aligned (swizzle atoms)
   uint8_t a[kStages][kABytes];
-  uint64_t c_full[kCStages];        // codes landed
-  uint64_t c_empty[kCStages];       // MMAs reading the codes stage done
-  uint64_t w_full[kStages];         // packed weights landed
-  uint64_t aready[kStages];         // converters wrote the TMEM A stage
-  uint64_t w_empty[kStages];        // MMAs reading the A stage (and the weights smem) done
+  uint64_t full[kStages];
+  uint64_t aready[kStages];
+  uint64_t empty[kStages];
   uint64_t done;
   uint32_t tmem_base;
   int abort;
@@ -188,11 +185,6 @@ HBL_DEVINL uint64_t smem_desc_sw128(uint32_t saddr) {
 
 // OUT_BF16: Y = bf16((D - csum) * s * alpha); else acc (int32) = D - csum.
 // map_codes loads 256-token boxes, map_codes_half 128-token boxes (split tiles).
-// The codes move in 128-k stages through a ring of six, the packed weights in
-// 256-k stages through a ring of four (one TMEM A stage each): the copy of a
-// code stage is issued five MMA half-stages (~2.5K cycles at the tensor pipe's
-// rate) before it is needed, which covers the L2-to-SM latency of a 32 KB copy;
-// with 64 KB code stages in a ring of three the window was two stages.
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_constant__ CUtensorMap map_codes_half,
@@ -204,20 +196,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int n0, m0, toks;
   cta_tile(blockIdx.x, full, (N + kRows - 1) / kRows, &n0, &m0, &toks);
-  const uint32_t cbytes = (uint32_t)toks * 128u;     // codes bytes per 128-k stage
+  const int bbytes = toks * kKBlock;                 // codes bytes per stage
   const uint32_t idesc = idesc_for(toks);
   const int nblk = K / kKBlock;
   volatile int* abort = &S.abort;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kCStages; ++s) {
-      mbar_init(&S.c_full[s], 1);
-      mbar_init(&S.c_empty[s], 1);
-    }
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&S.w_full[s], 1);
+      mbar_init(&S.full[s], 1);
       mbar_init(&S.aready[s], 128);
-      mbar_init(&S.w_empty[s], 1);
+      mbar_init(&S.empty[s], 1);
     }
     mbar_init(&S.done, 1);
     S.abort = 0;
@@ -233,39 +221,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
+  // number of stages the producer issued / MMAs committed (for the bounded drain on abort)
+  int issued = 0;
 
   if (warp == 0) {
     if (lane == 0) {
-      // issue order: weights of block kb, then its two code halves
-      const CUtensorMap* mc = toks == kToks ? &map_codes : &map_codes_half;
-      int wi = 0, ci = 0;   // weight / code stages issued
-      bool ok = true;
-      for (int kb = 0; kb < nblk && ok; ++kb) {
-        const int ws = kb % kStages;
-        if (kb >= kStages && !mbar_wait(&S.w_empty[ws], ((uint32_t)(kb / kStages) & 1u) ^ 1u, abort)) break;
-        mbar_expect_tx(&S.w_full[ws], (uint32_t)kABytes);
-        tma_load_2d(&S.a[ws][0], &map_w, &S.w_full[ws], kb * (kKBlock / 4), n0);
-        wi = kb + 1;
-        for (int h = 0; h < 2; ++h) {
-          const int c = 2 * kb + h, cs = c % kCStages;
-          if (c >= kCStages && !mbar_wait(&S.c_empty[cs], ((uint32_t)(c / kCStages) & 1u) ^ 1u, abort)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(&S.c_full[cs], cbytes);
-          tma_load_2d(&S.b[cs][0], mc, &S.c_full[cs], kb * kKBlock + 128 * h, m0);
-          ci = c + 1;
-        }
+      for (int kb = 0; kb < nblk; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+        if (kb >= kStages && !mbar_wait(&S.empty[s], ph ^ 1u, abort)) break;
+        const CUtensorMap* mc = toks == kToks ? &map_codes : &map_codes_half;
+        mbar_expect_tx(&S.full[s], (uint32_t)(bbytes + kABytes));
+        tma_load_2d(&S.b[s][0], mc, &S.full[s], kb * kKBlock, m0);
+        tma_load_2d(&S.b[s][bbytes / 2], mc, &S.full[s], kb * kKBlock + 128, m0);
+        tma_load_2d(&S.a[s][0], &map_w, &S.full[s], kb * (kKBlock / 4), n0);
+        ++issued;
       }
       // drain: wait (bounded) for the last loads issued to land before anyone may exit
-      for (int q = (wi > kStages ? wi - kStages : 0); q < wi; ++q) {
+      for (int kb = (issued > kStages ? issued - kStages : 0); kb < issued; ++kb) {
+        const int s = kb % kStages;
         const long long t0 = clock64();
-        while (!mbar_try_wait(&S.w_full[q % kStages], (uint32_t)(q / kStages) & 1u) && clock64() - t0 < kSpinLimit) {
-        }
-      }
-      for (int q = (ci > kCStages ? ci - kCStages : 0); q < ci; ++q) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&S.c_full[q % kCStages], (uint32_t)(q / kCStages) & 1u) && clock64() - t0 < kSpinLimit) {
+        while (!mbar_try_wait(&S.full[s], (uint32_t)(kb / kStages) & 1u) && clock64() - t0 < kSpinLimit) {
         }
       }
     }
@@ -273,22 +249,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
     if (lane == 0) {
       bool ok = true;
       for (int kb = 0; kb < nblk && ok; ++kb) {
-        const int ws = kb % kStages;
-        if (!mbar_wait(&S.aready[ws], (uint32_t)(kb / kStages) & 1u, abort)) break;
-        for (int h = 0; h < 2; ++h) {
-          const int c = 2 * kb + h, cs = c % kCStages;
-          if (!mbar_wait(&S.c_full[cs], (uint32_t)(c / kCStages) & 1u, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t bbase = su32(&S.b[cs][0]);
+        const int s = kb % kStages;
+        const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
+        ok = mbar_wait(&S.full[s], ph, abort) && mbar_wait(&S.aready[s], ph, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t bbase = su32(&S.b[s][0]);
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const int j = 4 * h + jj;
-            const uint32_t a_addr = tmem + (uint32_t)(kDCols + ws * kACols + 8 * j);
-            mma_i8_ts(tmem, a_addr, smem_desc_sw128(bbase + (uint32_t)(jj * 32)), idesc, (kb > 0 || j > 0) ? 1u : 0u);
-          }
-          tc_commit(&S.c_empty[cs]);
+        for (int j = 0; j < kKBlock / 32; ++j) {
+          const uint32_t a_addr = tmem + (uint32_t)(kDCols + s * kACols + 8 * j);
+          const uint64_t bdesc = smem_desc_sw128(bbase + (uint32_t)((j >> 2) * (bbytes / 2) + (j & 3) * 32));
+          mma_i8_ts(tmem, a_addr, bdesc, idesc, (kb > 0 || j > 0) ? 1u : 0u);
         }
-        if (ok) tc_commit(&S.w_empty[ws]);
+        tc_commit(&S.empty[s]);
+        ++issued;
       }
       tc_commit(&S.done);   // arrives once every MMA issued above has completed
     }
@@ -300,10 +274,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
     for (int kb = 0; kb < nblk; ++kb) {
       const int s = kb % kStages;
       const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      // the weight stage landed, and (it is only reloaded once) the MMAs of its
-      // previous use are done, so its TMEM A stage is free
-      if (!__all_sync(0xffffffffu, mbar_wait(&S.w_full[s], ph, abort))) break;
-      tc_fence_after();
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], ph, abort))) break;
       // the tile arrives 64B-swizzled: 16-byte chunk t of row `row` sits at
       // chunk t ^ ((row >> 1) & 3), which spreads a quarter-warp's 8 rows over
       // all 32 banks

@@ -233,7 +233,6 @@ struct FwhtArgs {
   float* scales;
   int32_t* csum;
   float* Xr;            // fp32 output (kModeF32)
-  int sm_count;         // SMs of the device (persistent configurations)
 };
 
 template <int LOG_K, int G, int MODE, bool IN_F32, bool LN>
@@ -245,47 +244,6 @@ void launch_fwht(const FwhtArgs& a, cudaStream_t s) {
   launch_pdl(fwht_quant_kernel<LOG_K, G, MODE, IN_F32, LN>, dim3(grid), dim3(C::THREADS), C::SMEM, s, a.X, a.M,
              a.gain, a.codes, a.scales, a.csum, a.Xr);
 }
-
-// CTAs of `kern` resident per SM at `threads` threads and `smem` bytes (cached per device and kernel).
-template <typename F>
-int blocks_per_sm(F* kern, int threads, size_t smem) {
-  struct Entry { int dev; const void* fn; int n; };
-  static std::mutex mu;
-  static std::vector<Entry> known;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lk(mu);
-  for (auto& e : known)
-    if (e.dev == dev && e.fn == (const void*)kern) return e.n;
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess || n < 1) {
-    (void)cudaGetLastError();
-    n = 1;
-  }
-  known.push_back(Entry{dev, (const void*)kern, n});
-  return n;
-}
-
-// The persistent Hadamard kernel: as many CTAs as fit on the device at once
-// (never more than there are tokens), each walking tokens with a stride of the grid.
-template <int LOG_K, int G, int MODE, bool IN_F32, bool LN, bool STAGED>
-void launch_fwht_persist(const FwhtArgs& a, cudaStream_t s) {
-  using C = FwhtCfg<LOG_K, G>;
-  auto* kern = fwht_quant_persist_kernel<LOG_K, G, MODE, IN_F32, LN, STAGED>;
-  const size_t smem = C::SMEM + (STAGED ? (size_t)C::K * (IN_F32 ? 4 : 2) : 0);
-  ensure_smem_attr(kern, smem);
-  const long long cap = (long long)blocks_per_sm(kern, C::THREADS, smem) * a.sm_count;
-  const int grid = (int)(a.M < cap ? a.M : cap);
-  ProfScope ps("fwht_quant", s);
-  launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, s, a.X, a.M, a.gain, a.codes, a.scales, a.csum, a.Xr);
-}
-
-// Many-token form of the K = 16384 transform: 0 = one token per CTA (grid of
-// M CTAs), 1 = persistent with a staging buffer, 2 = persistent, row fetched
-// into the exchange buffer.
-#ifndef HBL_FWHT_PERSIST
-#define HBL_FWHT_PERSIST 0
-#endif
 
 constexpr int kLatencyTokens = 64;
 
@@ -312,11 +270,7 @@ int dispatch_fwht(const FwhtArgs& a, int K, cudaStream_t s) {
     case 11: launch_fwht<11, 6, MODE, IN_F32, LN>(a, s); break;
     case 12: launch_fwht<12, 6, MODE, IN_F32, LN>(a, s); break;
     case 13: launch_fwht<13, 7, MODE, IN_F32, LN>(a, s); break;
-    case 14:
-      if (HBL_FWHT_PERSIST == 1) launch_fwht_persist<14, 7, MODE, IN_F32, LN, true>(a, s);
-      else if (HBL_FWHT_PERSIST == 2) launch_fwht_persist<14, 7, MODE, IN_F32, LN, false>(a, s);
-      else launch_fwht<14, 7, MODE, IN_F32, LN>(a, s);
-      break;
+    case 14: launch_fwht<14, 7, MODE, IN_F32, LN>(a, s); break;
     case 15: launch_fwht<15, 5, MODE, IN_F32, LN>(a, s); break;
     default: return HBL_ERR_SHAPE;
   }
@@ -352,9 +306,8 @@ int dispatch_rows(const uint16_t* X, int M, int K, const float* gain, int8_t* co
 
 // Optional RMSNorm (ln), optional Hadamard, then the per-token quantiser.
 int run_quantize(const uint16_t* X, int M, int K, int act_bits, int use_hadamard, int8_t* codes,
-                 float* scales, int32_t* csum, int sm_count, cudaStream_t s, bool ln = false,
-                 const float* gain = nullptr) {
-  const FwhtArgs a{X, M, gain, codes, scales, csum, nullptr, sm_count};
+                 float* scales, int32_t* csum, cudaStream_t s, bool ln = false, const float* gain = nullptr) {
+  const FwhtArgs a{X, M, gain, codes, scales, csum, nullptr};
   if (use_hadamard) {
     if (ln)
       return act_bits == 4 ? dispatch_fwht<kModeInt4, false, true>(a, K, s)
@@ -841,7 +794,7 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
     const int fs = run_fused_decode(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, ln, gain, Y, d->sm_count, s);
     if (fs != kFusedNotApplicable) return fs;
   }
-  int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, d->sm_count, s, ln, gain);
+  int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
   if (st) return st;
   switch (choose_gemm(M, K, N, path)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
@@ -984,7 +937,7 @@ int hbl_hadamard_f32(const hbl_bf16* X, int M, int K, float* Xr, hbl_stream stre
   if (misaligned16(X) || misaligned16(Xr)) return HBL_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   if ((st = ensure_device(&d))) return st;
-  return dispatch_fwht<kModeF32>(FwhtArgs{X, M, nullptr, nullptr, nullptr, nullptr, Xr, d->sm_count}, K,
+  return dispatch_fwht<kModeF32>(FwhtArgs{X, M, nullptr, nullptr, nullptr, nullptr, Xr}, K,
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -998,8 +951,7 @@ int hbl_quantize(const hbl_bf16* X, int M, int K, int act_bits, int use_hadamard
   if (misaligned16(X) || misaligned16(codes)) return HBL_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   if ((st = ensure_device(&d))) return st;
-  return run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, d->sm_count,
-                      reinterpret_cast<cudaStream_t>(stream));
+  return run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, int32_t* acc, hbl_stream stream) {
@@ -1064,8 +1016,8 @@ int hbl_quantize_ln(const hbl_bf16* X, int M, int K, const float* gain, int act_
   if (misaligned16(X) || misaligned16(codes) || misaligned16(gain)) return HBL_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   if ((st = ensure_device(&d))) return st;
-  return run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, d->sm_count,
-                      reinterpret_cast<cudaStream_t>(stream), true, gain);
+  return run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, reinterpret_cast<cudaStream_t>(stream),
+                      true, gain);
 }
 
 int hbl_hadamard_backward_f32(const float* dXr, int M, int K, float* dX, hbl_stream stream) {
@@ -1075,7 +1027,7 @@ int hbl_hadamard_backward_f32(const float* dXr, int M, int K, float* dX, hbl_str
   if (misaligned16(dXr) || misaligned16(dX)) return HBL_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   if ((st = ensure_device(&d))) return st;
-  return dispatch_fwht<kModeF32, true, false>(FwhtArgs{dXr, M, nullptr, nullptr, nullptr, nullptr, dX, d->sm_count}, K,
+  return dispatch_fwht<kModeF32, true, false>(FwhtArgs{dXr, M, nullptr, nullptr, nullptr, nullptr, dX}, K,
                                               reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1089,7 +1041,7 @@ int hbl_pack_weights_rotated(const float* W, int N, int K, uint8_t* Wpk, float* 
   DeviceState* d = nullptr;
   if ((st = ensure_device(&d))) return st;
   // every weight row w becomes H w (W H^T), in fp32, then the usual ternarise + pack
-  st = dispatch_fwht<kModeF32, true, false>(FwhtArgs{W, N, nullptr, nullptr, nullptr, nullptr, Wrot, d->sm_count}, K,
+  st = dispatch_fwht<kModeF32, true, false>(FwhtArgs{W, N, nullptr, nullptr, nullptr, nullptr, Wrot}, K,
                                             reinterpret_cast<cudaStream_t>(stream));
   if (st) return st;
   return hbl_pack_weights(Wrot, N, K, Wpk, wscale, stream);
