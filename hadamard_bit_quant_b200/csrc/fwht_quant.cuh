@@ -55,27 +55,51 @@ HBL_DEVINL int pass_index(int t, int j, int lo) {
 template <int G, int PADW = 1>
 HBL_DEVINL int pad(int idx) { return idx + PADW * (idx >> G); }
 
+// Packed two-lane fp32 arithmetic of sm_100 (each lane an IEEE operation with
+// round-to-nearest-even, the same result as the scalar instruction).
+HBL_DEVINL float2 f2_add(float2 a, float2 b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+      "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+HBL_DEVINL float2 f2_sub(float2 a, float2 b) {
+  unsigned long long r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+      "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+HBL_DEVINL float2 f2_fma(float2 a, float2 b, float2 c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+      "l"(*reinterpret_cast<unsigned long long*>(&b)), "l"(*reinterpret_cast<unsigned long long*>(&c)));
+  return *reinterpret_cast<float2*>(&r);
+}
+
 // Codes of four values, RoundClip(mult * v, lo, hi) with round half to even,
-// packed little-endian into one word. The product is rounded to fp32 first;
-// with CLAMP it is clamped to the integral bounds [lo, hi] (clamping commutes
-// with rounding to an integer there); adding 1.5 * 2^23 then rounds it to an
-// integer whose two's-complement low byte is the low mantissa byte of the sum
-// (|x| < 2^22). Without CLAMP the caller guarantees |mult * v| < 127.5 (the
-// absmax quantiser: |v| <= gamma < gamma + eps).
+// packed little-endian into one word. One fused multiply-add per value forms
+// mult * v + 1.5 * 2^23 with a single rounding: for |mult * v| < 2^22 the sum
+// lies in [2^23, 2^24), where the float spacing is 1, so the rounding is the
+// round-half-to-even of the exact product mult * v to an integer n, and the
+// low mantissa byte of the sum is n's two's-complement low byte. With CLAMP
+// the sum is then clamped to [1.5 * 2^23 + lo, 1.5 * 2^23 + hi] (exact; a
+// product beyond +-2^22 lands outside that range and is clamped the same
+// way). Without CLAMP the caller guarantees |mult * v| < 127.5 (the absmax
+// quantiser: |v| <= gamma < gamma + eps).
 template <bool CLAMP>
 HBL_DEVINL uint32_t quant4(float v0, float v1, float v2, float v3, float mult, float lo, float hi) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
   const float2 m2 = make_float2(mult, mult);
-  float2 a = __fmul2_rn(make_float2(v0, v1), m2);
-  float2 b = __fmul2_rn(make_float2(v2, v3), m2);
+  const float2 magic = make_float2(kMagic, kMagic);
+  float2 a = f2_fma(make_float2(v0, v1), m2, magic);
+  float2 b = f2_fma(make_float2(v2, v3), m2, magic);
   if constexpr (CLAMP) {
-    a.x = fminf(fmaxf(a.x, lo), hi);
-    a.y = fminf(fmaxf(a.y, lo), hi);
-    b.x = fminf(fmaxf(b.x, lo), hi);
-    b.y = fminf(fmaxf(b.y, lo), hi);
+    const float l = kMagic + lo, h = kMagic + hi;
+    a.x = fminf(fmaxf(a.x, l), h);
+    a.y = fminf(fmaxf(a.y, l), h);
+    b.x = fminf(fmaxf(b.x, l), h);
+    b.y = fminf(fmaxf(b.y, l), h);
   }
-  const float2 magic = make_float2(12582912.0f, 12582912.0f);
-  a = __fadd2_rn(a, magic);
-  b = __fadd2_rn(b, magic);
   const uint32_t lo2 = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040);
   const uint32_t hi2 = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040);
   return __byte_perm(lo2, hi2, 0x5410);
@@ -154,12 +178,23 @@ HBL_DEVINL void quant_tail(float (&v)[E], int K, int t, int token_sub, bool acti
     return;
   } else {
     float part = 0.f;
-    if constexpr (MODE == kModeInt4) {
+    if constexpr (MODE == kModeInt4 && E >= 64) {
+      // many values per thread (configurations with no fused counterpart):
+      // eight interleaved partial sums, added in a fixed tree, instead of one
+      // chain of E dependent additions
+      float p8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < E; ++j) p8[j & 7] += fabsf(v[j]);
+      part = ((p8[0] + p8[1]) + (p8[2] + p8[3])) + ((p8[4] + p8[5]) + (p8[6] + p8[7]));
+    } else if constexpr (MODE == kModeInt4) {
 #pragma unroll
       for (int j = 0; j < E; ++j) part += fabsf(v[j]);
     } else {
+      // the maximum does not depend on the order: eight interleaved chains
+      float p8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < E; ++j) part = fmaxf(part, fabsf(v[j]));
+      for (int j = 0; j < E; ++j) p8[j & 7] = fmaxf(p8[j & 7], fabsf(v[j]));
+      part = fmaxf(fmaxf(fmaxf(p8[0], p8[1]), fmaxf(p8[2], p8[3])), fmaxf(fmaxf(p8[4], p8[5]), fmaxf(p8[6], p8[7])));
     }
     const float r = __fmul_rn(token_reduce_f<T, WPT, MODE == kModeInt8>(part, red_f, token_sub), nrm);
     float mult, scale;
@@ -225,8 +260,8 @@ HBL_DEVINL void butterflies(float (&v)[E], int nb) {
         const int k = j | (1 << r);
         const float2 a = make_float2(v[j], v[j + 1]);
         const float2 b = make_float2(v[k], v[k + 1]);
-        const float2 s = __fadd2_rn(a, b);
-        const float2 d = __fadd2_rn(a, make_float2(-b.x, -b.y));
+        const float2 s = f2_add(a, b);
+        const float2 d = f2_sub(a, b);
         v[j] = s.x; v[j + 1] = s.y;
         v[k] = d.x; v[k + 1] = d.y;
       }
