@@ -23,6 +23,7 @@ namespace hbl {
 
 enum QuantMode { kModeInt4 = 0, kModeInt8 = 1, kModeF32 = 2 };
 
+
 template <int LOG_K, int G>
 struct FwhtCfg {
   static constexpr int K = 1 << LOG_K;
@@ -296,7 +297,13 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
   constexpr uint32_t kRowBytes = (uint32_t)K * (IN_F32 ? 4u : 2u);
   const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&stage_bar);
 
-  if (threadIdx.x == 0) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(bar) : "memory");
+    // make the initialised barrier visible to the bulk-copy (async) proxy before
+    // a copy completes on it: without this, the copy may act on whatever barrier
+    // state an earlier CTA left at the same shared-memory address
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
   __syncthreads();
   // Programmatic dependent launch: let the consumer grid launch now (it only
   // prefetches weights until this grid completes), and wait for the producer
