@@ -49,7 +49,8 @@ static_assert(kDCols + kStages * kACols <= kTmemCols, "TMEM columns");
 struct __align__(8) Smem {
   uint8_t b[kStages][kBBytes];      // 1024-byte aligned (swizzle atoms)
   uint8_t a[kStages][kABytes];
-  uint64_t full[kStages];
+  uint64_t full[kStages];           // the stage's codes landed
+  uint64_t w_full[kStages];         // the stage's packed weights landed
   uint64_t aready[kStages];
   uint64_t empty[kStages];
   uint64_t done;
@@ -204,6 +205,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
+      mbar_init(&S.w_full[s], 1);
       mbar_init(&S.aready[s], 128);
       mbar_init(&S.empty[s], 1);
     }
@@ -231,10 +233,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
         const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
         if (kb >= kStages && !mbar_wait(&S.empty[s], ph ^ 1u, abort)) break;
         const CUtensorMap* mc = toks == kToks ? &map_codes : &map_codes_half;
-        mbar_expect_tx(&S.full[s], (uint32_t)(bbytes + kABytes));
+        // the weights first, on their own barrier: the converters unpack them
+        // while the codes are still arriving
+        mbar_expect_tx(&S.w_full[s], (uint32_t)kABytes);
+        tma_load_2d(&S.a[s][0], &map_w, &S.w_full[s], kb * (kKBlock / 4), n0);
+        mbar_expect_tx(&S.full[s], (uint32_t)bbytes);
         tma_load_2d(&S.b[s][0], mc, &S.full[s], kb * kKBlock, m0);
         tma_load_2d(&S.b[s][bbytes / 2], mc, &S.full[s], kb * kKBlock + 128, m0);
-        tma_load_2d(&S.a[s][0], &map_w, &S.full[s], kb * (kKBlock / 4), n0);
         ++issued;
       }
       // drain: wait (bounded) for the last loads issued to land before anyone may exit
@@ -242,6 +247,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
         const int s = kb % kStages;
         const long long t0 = clock64();
         while (!mbar_try_wait(&S.full[s], (uint32_t)(kb / kStages) & 1u) && clock64() - t0 < kSpinLimit) {
+        }
+        while (!mbar_try_wait(&S.w_full[s], (uint32_t)(kb / kStages) & 1u) && clock64() - t0 < kSpinLimit) {
         }
       }
     }
@@ -274,7 +281,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_codes, const __grid_const
     for (int kb = 0; kb < nblk; ++kb) {
       const int s = kb % kStages;
       const uint32_t ph = (uint32_t)(kb / kStages) & 1u;
-      if (!__all_sync(0xffffffffu, mbar_wait(&S.full[s], ph, abort))) break;
+      // the weights landed; the producer reloads a stage only once its
+      // previous MMAs are done, so its TMEM A stage is free
+      if (!__all_sync(0xffffffffu, mbar_wait(&S.w_full[s], ph, abort))) break;
+      tc_fence_after();
       // the tile arrives 64B-swizzled: 16-byte chunk t of row `row` sits at
       // chunk t ^ ((row >> 1) & 3), which spreads a quarter-warp's 8 rows over
       // all 32 banks
