@@ -16,7 +16,6 @@
 #include "gemm_mma.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
-#include "gemm_tcw.cuh"
 #include "gemm_decode.cuh"
 #include "gemm_decode2.cuh"
 #include "gemm_stream.cuh"
@@ -412,8 +411,7 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 // 0 auto, 1 warp-level mma.sync, 2 tcgen05 persistent (128 x 128 tiles), 3 decode without
 // clusters or streaming, 4 tcgen05 one 128 x 256 tile per CTA (the default for M >= 128),
 // 5 weight-streaming decode (the default for M <= 16 where it fits), 6 as 0 (the forward
-// takes the fused single-kernel decode wherever it fits; 0 does the same), 7 tcgen05
-// persistent with 256 x 128 tiles.
+// takes the fused single-kernel decode wherever it fits; 0 does the same).
 // Every entry point reads it once and passes the value down, so one call never
 // mixes two settings.
 std::atomic<int> g_gemm_path{0};
@@ -474,36 +472,11 @@ int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, co
   return launch_status();
 }
 
-// Persistent tcgen05 kernel with 256 weight rows x 128 tokens per tile (each
-// code tile in shared memory feeds two M=128 MMAs).
-int run_gemm_tcw(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, const int32_t* csum,
-                 const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count,
-                 cudaStream_t s) {
-  CUtensorMap mc, mw;
-  if (!make_map_u8(&mc, codes, (uint64_t)K, (uint64_t)M, (uint64_t)K, 128, tcw::kToks, 128)) return HBL_ERR_CUDA;
-  if (!make_map_u8(&mw, Wpk, (uint64_t)K / 4, (uint64_t)N, (uint64_t)K / 4, kKBlock / 4, tcw::kRows, 64))
-    return HBL_ERR_CUDA;
-  const int tiles = ((N + tcw::kRows - 1) / tcw::kRows) * ((M + tcw::kToks - 1) / tcw::kToks);
-  const dim3 grid(tiles < sm_count ? tiles : sm_count);
-  ProfScope ps("gemm_tc", s);
-  cudaError_t e;
-  if (Y) {
-    ensure_smem_attr(tcw::gemm_tcw_kernel<true>, tcw::kSmemBytes);
-    e = launch_pdl(tcw::gemm_tcw_kernel<true>, grid, dim3(tcw::kThreads), tcw::kSmemBytes, s, mc, mw, M, K, N,
-                   csum, scales, alpha, Y, (int32_t*)nullptr);
-  } else {
-    ensure_smem_attr(tcw::gemm_tcw_kernel<false>, tcw::kSmemBytes);
-    e = launch_pdl(tcw::gemm_tcw_kernel<false>, grid, dim3(tcw::kThreads), tcw::kSmemBytes, s, mc, mw, M, K, N,
-                   csum, (const float*)nullptr, (const float*)nullptr, (uint16_t*)nullptr, acc);
-  }
-  return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
-}
-
 bool decode_path_fits(int M, int K) {
   return M <= kLatencyTokens && dec::smem_bytes(K, 8) <= 200 * 1024;
 }
 
-enum class GemmKind { Decode, Mma, Tc, Tc2, Tcw };
+enum class GemmKind { Decode, Mma, Tc, Tc2 };
 
 // Which GEMM kernel runs (after the quantiser). By size, from timings on B200
 // over M in 1..4096 and K, N in 2048..16384:
@@ -520,7 +493,6 @@ GemmKind choose_gemm(int M, int K, int N, int path) {
     case 1: return GemmKind::Mma;
     case 2: return GemmKind::Tc2;
     case 4: return GemmKind::Tc;
-    case 7: return GemmKind::Tcw;
     default: break;
   }
   if (M <= 16 && decode_path_fits(M, K)) return GemmKind::Decode;
@@ -799,7 +771,6 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   switch (choose_gemm(M, K, N, path)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
     case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
-    case GemmKind::Tcw: return run_gemm_tcw(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, d->sm_count, s);
     case GemmKind::Decode:
       return run_gemm_decode(codes, M, K, N, Wpk, csum, scales, wscale, Y, nullptr, s, d->sm_count, path);
     case GemmKind::Mma: break;
@@ -984,7 +955,6 @@ int hbl_gemm_codes(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk,
   switch (choose_gemm(M, K, N, path)) {
     case GemmKind::Tc2: return run_gemm_tc2(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
     case GemmKind::Tc: return run_gemm_tc(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
-    case GemmKind::Tcw: return run_gemm_tcw(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, d->sm_count, s);
     case GemmKind::Decode:
       return run_gemm_decode(codes, M, K, N, Wpk, csum, nullptr, nullptr, nullptr, acc, s, d->sm_count, path);
     case GemmKind::Mma: break;
@@ -1070,7 +1040,7 @@ int hbl_quantize_qkv(const hbl_bf16* X, int T, int H, int d, int bits, int bos_t
 }
 
 int hbl_set_gemm_path(int path) {
-  if (path < 0 || path > 7) return HBL_ERR_INVALID_ARG;
+  if (path < 0 || path > 6) return HBL_ERR_INVALID_ARG;
   g_gemm_path.store(path, std::memory_order_relaxed);
   return HBL_OK;
 }

@@ -284,14 +284,13 @@ int hbl_get_device_error(hbl_stream stream);
  * 1 = always the warp-level split-K kernel, 2 = always the persistent tcgen05
  * kernel, 3 = as 0 but never the fused, cluster or streaming decode kernels,
  * 4 = always the one-tile tcgen05 kernel, 5 = as 0 but never the fused
- * forward, 6 = as 0, 7 = always the persistent tcgen05 kernel with 256 weight
- * rows x 128 tokens per tile.
+ * forward, 6 = as 0.
  * All give results within the parity bounds of the oracle (the fused forward
  * and the quantiser kernel share their summation order, so the paths give the
  * same bits); the knob exists to check and time each one. Process-wide; each
  * forward or hbl_gemm_codes call reads it once when it starts, so a change
  * made while calls run on other threads applies from their next call on.
- * Returns HBL_ERR_INVALID_ARG for a value outside 0..7.
+ * Returns HBL_ERR_INVALID_ARG for a value outside 0..6.
  */
 int hbl_set_gemm_path(int path);
 

@@ -65,10 +65,10 @@ def test_gemm_path_selector_bounds(lib):
     from hadamard_bit_quant_b200 import hbl
     raw = hbl.lib()
     try:
-        for p in range(8):
+        for p in range(7):
             assert raw.hbl_set_gemm_path(p) == 0
         assert raw.hbl_set_gemm_path(-1) == 1
-        assert raw.hbl_set_gemm_path(8) == 1
+        assert raw.hbl_set_gemm_path(7) == 1
     finally:
         assert raw.hbl_set_gemm_path(0) == 0
 
