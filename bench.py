@@ -145,12 +145,12 @@ class ClockSampler:
 
 class ClockPoller:
     """SM clock and clock-event (throttle) reasons read through NVML from a background
-    thread every ~0.5 ms while running: read-only queries, fine-grained enough for a timed
-    region of a few milliseconds (nvidia-smi samples every 200 ms at best)."""
+    thread, back to back, while running: read-only queries, as fine-grained as NVML allows
+    for a timed region of a few milliseconds (nvidia-smi samples every 200 ms at best)."""
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, torch, local, period_s=0.0005):
+    def __init__(self, torch, local, period_s=0.0):
         self.torch, self.local, self.period = torch, local, period_s
         self.samples, self.thread, self.h, self.nv = [], None, None, None
         self.stop_flag = False
@@ -177,7 +177,8 @@ class ClockPoller:
                 self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), self._reasons()))
             except Exception:
                 pass
-            time.sleep(self.period)
+            if self.period > 0:
+                time.sleep(self.period)
 
     def start(self):
         import threading
@@ -205,7 +206,7 @@ class ClockPoller:
         return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": float(self.smax),
                 "reasons": sorted(reasons), "samples": len(self.samples),
                 "sm_mhz_min": min(c for c, _ in self.samples),
-                "source": "NVML clock and clock-event reasons polled every 0.5 ms during the timed region"}
+                "source": "NVML clock and clock-event reasons polled back to back during the timed region"}
 
 
 # ----------------------------------------------------------------------------- workloads
