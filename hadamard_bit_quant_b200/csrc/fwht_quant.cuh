@@ -353,7 +353,34 @@ fwht_quant_kernel(const void* __restrict__ Xv, int M, const float* __restrict__ 
 #pragma unroll
     for (int j = 0; j < E; ++j) v[j] = 0.f;
   }
-  if constexpr (LN) {
+  if constexpr (LN && E >= 64) {
+    // Many values per thread (no fused counterpart): the sum of squares of
+    // the raw values runs as eight interleaved chains and is finished before
+    // any gain is applied; the gain loads take their address from an opaque
+    // zero computed from it, and then from each group's last product, 16
+    // values at a time. Otherwise the compiler keeps every raw value alive for
+    // the sum while it forms the gain products early, doubling the live values
+    // (255 registers and spills). The products are the same whatever the schedule.
+    float q8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < E; ++j) q8[j & 7] = __fmaf_rn(v[j], v[j], q8[j & 7]);
+    ssq = ((q8[0] + q8[1]) + (q8[2] + q8[3])) + ((q8[4] + q8[5]) + (q8[6] + q8[7]));
+    if (gain) {
+      uint32_t z;
+      asm volatile("and.b32 %0, %1, 0;\n" : "=r"(z) : "r"(__float_as_uint(ssq)));
+      const float* gp = gain + t + z;
+#pragma unroll
+      for (int j0 = 0; j0 < E; j0 += 16) {
+        float g[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) g[i] = __ldg(gp + (j0 + i) * T);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[j0 + i] = __fmul_rn(v[j0 + i], g[i]);
+        asm volatile("and.b32 %0, %1, 0;\n" : "=r"(z) : "r"(__float_as_uint(v[j0 + 15])));
+        gp += z;
+      }
+    }
+  } else if constexpr (LN) {
 #pragma unroll
     for (int j = 0; j < E; ++j) ssq = __fmaf_rn(v[j], v[j], ssq);
     if (gain) {

@@ -26,25 +26,57 @@ HBL_DEVINL void add128(unsigned long long& lo, unsigned long long& hi, unsigned 
   lo = n;
 }
 
+// Adds |w| (an fp32 bit pattern) to the thread's exact accumulators: most
+// weights of a tensor share one exponent bucket, so a thread first tries the
+// bucket of its previous value (one compare, one 128-bit add) and only else
+// walks the eight buckets.
+HBL_DEVINL void abs_acc_add(uint32_t bits, unsigned long long (&lo)[8], unsigned long long (&hi)[8], int& hot,
+                            unsigned long long& hlo, unsigned long long& hhi, bool& bad) {
+  bits &= 0x7fffffffu;
+  uint32_t e = bits >> 23;
+  uint32_t m = bits & 0x7fffffu;
+  if (e == 255u) { bad = true; return; }
+  if (e) m |= 0x800000u; else e = 1u;
+  const int bkt = (int)(e >> 5);
+  const unsigned long long v = ((unsigned long long)m) << (e & 31u);
+  if (bkt == hot) {
+    add128(hlo, hhi, v);
+    return;
+  }
+  // flush the hot bucket into its slot and make this one hot
+#pragma unroll
+  for (int b = 0; b < 8; ++b)
+    if (hot == b) { add128(lo[b], hi[b], hlo); hi[b] += hhi; }
+  hot = bkt;
+  hlo = v;
+  hhi = 0ull;
+}
+
 __global__ void __launch_bounds__(256) abs_sum_kernel(const float* __restrict__ W, long long n,
                                                       AbsSumAcc* __restrict__ acc) {
   unsigned long long lo[8], hi[8];
 #pragma unroll
   for (int b = 0; b < 8; ++b) { lo[b] = 0ull; hi[b] = 0ull; }
+  int hot = -1;
+  unsigned long long hlo = 0ull, hhi = 0ull;
   bool bad = false;
   const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-    uint32_t bits = __float_as_uint(__ldg(W + i)) & 0x7fffffffu;
-    uint32_t e = bits >> 23;
-    uint32_t m = bits & 0x7fffffu;
-    if (e == 255u) { bad = true; continue; }
-    if (e) m |= 0x800000u; else e = 1u;
-    const uint32_t bkt = e >> 5;
-    const unsigned long long v = ((unsigned long long)m) << (e & 31u);
-#pragma unroll
-    for (int b = 0; b < 8; ++b)
-      if (bkt == (uint32_t)b) add128(lo[b], hi[b], v);
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if ((reinterpret_cast<uintptr_t>(W) & 15u) == 0 && (n & 3) == 0) {
+    const uint4* W4 = reinterpret_cast<const uint4*>(W);
+    for (long long i = tid; i < n / 4; i += stride) {
+      const uint4 q = __ldg(W4 + i);
+      abs_acc_add(q.x, lo, hi, hot, hlo, hhi, bad);
+      abs_acc_add(q.y, lo, hi, hot, hlo, hhi, bad);
+      abs_acc_add(q.z, lo, hi, hot, hlo, hhi, bad);
+      abs_acc_add(q.w, lo, hi, hot, hlo, hhi, bad);
+    }
+  } else {
+    for (long long i = tid; i < n; i += stride) abs_acc_add(__float_as_uint(__ldg(W + i)), lo, hi, hot, hlo, hhi, bad);
   }
+#pragma unroll
+  for (int b = 0; b < 8; ++b)
+    if (hot == b) { add128(lo[b], hi[b], hlo); hi[b] += hhi; }
   if (bad) set_device_error(HBL_ERR_INVALID_ARG);
   // warp reduction of each 128-bit bucket
 #pragma unroll
