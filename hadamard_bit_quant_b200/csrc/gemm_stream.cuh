@@ -6,20 +6,28 @@
 //
 // With few tokens the forward moves N*K/4 bytes of packed weights and little
 // else, so the kernel is built to keep HBM busy:
-//   * one CTA per SM (persistent); CTA c owns the 16-row groups c, c+G, ...
-//     over the whole of K, so no partial sums ever leave the CTA;
+//   * one CTA per SM (persistent); each CTA owns a contiguous run of 16-row
+//     groups (the runs differ by at most one group) over the whole of K, so no
+//     partial sums ever leave the CTA;
 //   * K is walked in chunks of 2048; a chunk's codes (M x 2048 int8) sit in
-//     one of two shared-memory buffers, one bulk copy per token row;
-//   * the weights of each (chunk, group) unit -- 16 rows x 512 bytes -- stream
-//     through a 16-stage ring (128 KB in flight per SM), one 3-D TMA copy per
-//     unit laid out as eight [16 rows][64 B] tiles. The ring is
-//     filled before the kernel waits for the quantiser grid (programmatic
+//     one of two shared-memory buffers, brought by ONE 3-D TMA copy (sixteen
+//     128B-swizzled [token][128 B] tiles; token rows past M read as zeros):
+//     a copy costs the TMA unit a few hundred cycles whatever its size, and
+//     one copy per token row left the unit, not HBM, setting the pace;
+//   * the weights stream in units of two neighbouring groups and one chunk --
+//     32 rows x 512 bytes, one 16 KB 3-D TMA copy laid out as eight
+//     [32 rows][64 B] tiles (an odd last group: one 8 KB copy of [16][64 B]
+//     tiles) -- through a ring of 10 (two token tiles) or 12 (one) slots,
+//     160 or 192 KB, as much as shared memory holds beside the codes. Copies of
+//     8 KB left the copy unit's fixed cost per copy setting the pace. The ring
+//     is filled before the kernel waits for the quantiser grid (programmatic
 //     dependent launch), so a layer's weights arrive while the previous
 //     kernel still runs;
 //   * 8 consumer warps take one 256-k block of each unit each: weights as the
-//     m16n8k32 A operand (u = t + 1 unpacked in registers), codes as B, both
-//     read free of bank conflicts, accumulating in
-//     registers across chunks; a dedicated producer warp issues the copies;
+//     m16n8k32 A operand (u = t + 1 unpacked in registers, read free of bank
+//     conflicts), codes as B (read step by step, at most a 2-way conflict),
+//     accumulating in registers across chunks; a dedicated producer warp
+//     issues the copies, weights two chunks ahead of the consumers;
 //   * at the end the 8 warps' partial sums are added in shared memory, the
 //     code sums subtracted, scaled and stored as bf16 (or int32).
 // Every mbarrier wait is bounded; a CTA that gives up sets the device error
@@ -37,11 +45,8 @@ constexpr int kChunk = 2048;                       // k per chunk
 constexpr int kBlocksPerChunk = kChunk / kKBlock;  // 8 = one per consumer warp
 constexpr int kConsumers = 8;
 constexpr int kThreads = 32 * (kConsumers + 1);
-#ifndef HBL_STREAM_STAGES
-#define HBL_STREAM_STAGES 16
-#endif
-constexpr int kStages = HBL_STREAM_STAGES;
-constexpr int kUnitBytes = kGroupRows * (kChunk / 4);   // 8 KB: 4 boxes of [16][128 B]
+constexpr int kGroupBytes = kGroupRows * (kChunk / 4);  // 8 KB: one group's chunk of weights
+constexpr int kUnitBytes = 2 * kGroupBytes;             // ring slot: two groups
 constexpr int kMaxGroups = 8;                      // per CTA
 constexpr long long kSpinLimit = 4000000000ll;
 
@@ -93,47 +98,37 @@ HBL_DEVINL void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, in
       "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
-// Contiguous global -> shared copy of `bytes` (multiple of 16, both ends 16-byte aligned).
-HBL_DEVINL void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
-                   su32(dst)),
-               "l"(src), "r"(bytes), "r"(su32(bar))
-               : "memory");
-}
-HBL_DEVINL void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];\n" ::"r"(
-          su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
 
-// One chunk of codes: MT token rows of kChunk bytes, row stride kChunk + 32
-// (each token row arrives by one bulk copy). The 32-byte pad puts rows m and
-// m + 1 four banks apart, so an m16n8k32 fragment read (each half-warp: 4
-// tokens x 32 bytes) touches 16 distinct 8-byte bank slots.
+// One chunk of codes: kChunk / 128 column tiles of [MT tokens][128 B], each
+// 128B-swizzled (16-byte unit u of token row m at u ^ (m & 7)). A fragment
+// read (half-warp: 4 tokens x 32 bytes) meets at most a 2-way bank conflict;
+// it happens once per chunk and serves every unit of the chunk.
 template <int MT>
 struct Layout {
-  static constexpr int kCodeRow = kChunk + 32;
-  static constexpr int kCodeBuf = MT * kCodeRow;
+  static constexpr int kStages = MT == 8 ? 12 : 10;       // weight ring slots
+  static constexpr int kCodeTile = MT * 128;
+  static constexpr int kCodeBuf = (kChunk / 128) * kCodeTile;
   static constexpr size_t kRing = (size_t)kStages * kUnitBytes;
   // wfull, wempty [kStages]; cfull, cempty [2]; abort flag
   static constexpr size_t kBarBytes = (size_t)(2 * kStages + 4) * 8 + 16;
   static constexpr size_t kBytes = 1024 + kRing + 2 * (size_t)kCodeBuf + kBarBytes;
+  static_assert(kBytes <= 227 * 1024, "shared memory per block");
 };
 
-// Consumer side for a CTA that owns exactly NG groups: per chunk, wait for
-// the chunk's codes and all NG weight units, load every fragment, release the
-// slots, then issue the chunk's MMAs q by q over all groups (2*NG independent
-// accumulator chains; with one token tile, even and odd q accumulate
-// separately). The NG unit barriers are probed back to back with test_wait
-// (non-blocking), so their round trips (on the order of a hundred cycles
-// each) overlap; only a unit still in flight is waited for. Ends by writing this warp's partial sums into shared memory
+// Consumer side for a CTA that owns exactly NG groups (NU = ceil(NG / 2)
+// units per chunk; group b sits in unit b / 2, rows 16 * (b % 2) on): per
+// chunk, wait for the chunk's codes and all NU weight units, load every
+// fragment, release the slots, then issue the chunk's MMAs q by q over all
+// groups (2*NG independent accumulator chains; with one token tile, even and
+// odd q accumulate separately). The unit barriers are probed back to back with
+// test_wait (non-blocking), so their round trips (on the order of a hundred
+// cycles each) overlap; only a unit still in flight is waited for. Ends by writing this warp's partial sums into shared memory
 // (aliasing the ring) once every consumer warp is past its last unit.
 template <int NG, int TN, int MT>
 HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_t* wfull, uint64_t* wempty,
                         uint64_t* cfull, uint64_t* cempty, volatile int* abort, int warp, int lane) {
   using Lay = Layout<MT>;
+  constexpr int kStages = Lay::kStages;
   constexpr int SPLIT = TN == 1 ? 2 : 1;
   const int g = lane >> 2, tig = lane & 3;
   int acc[NG][TN * SPLIT][4];
@@ -147,32 +142,29 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
   for (int c = 0; c < nchunks && ok; ++c) {
     if (!__all_sync(0xffffffffu, mbar_wait(&cfull[c & 1], (uint32_t)(c >> 1) & 1u, abort))) { ok = false; break; }
     const uint8_t* cb = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
-    uint2 bf[TN][8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-#pragma unroll
-      for (int i = 0; i < TN; ++i) {
-        const int m = 8 * i + g;   // k = 256 * warp + 32 * q + 8 * tig .. + 7 of the chunk
-        bf[i][q] = *reinterpret_cast<const uint2*>(cb + m * Lay::kCodeRow + 256 * warp + 32 * q + 8 * tig);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
+    constexpr int NU = (NG + 1) / 2;
     uint32_t A4[NG][4], B4[NG][4];
-    bool landed[NG];
+    bool landed[NU];
 #pragma unroll
-    for (int b = 0; b < NG; ++b) {
-      const int u = c * NG + b;
-      landed[b] = mbar_test(&wfull[u % kStages], (uint32_t)(u / kStages) & 1u);
+    for (int v = 0; v < NU; ++v) {
+      const int u = c * NU + v;
+      landed[v] = mbar_test(&wfull[u % kStages], (uint32_t)(u / kStages) & 1u);
+    }
+#pragma unroll
+    for (int v = 0; v < NU; ++v) {
+      const int u = c * NU + v;
+      if (!__all_sync(0xffffffffu, landed[v] || mbar_wait(&wfull[u % kStages], (uint32_t)(u / kStages) & 1u, abort)))
+        ok = false;
     }
 #pragma unroll
     for (int b = 0; b < NG; ++b) {
-      const int u = c * NG + b;
-      const int s = u % kStages;
-      if (!__all_sync(0xffffffffu, landed[b] || mbar_wait(&wfull[s], (uint32_t)(u / kStages) & 1u, abort))) ok = false;
-      // block `warp` of the unit: tile `warp`, [16 rows][64 B]; rows 64 B apart,
+      const int v = b >> 1;
+      const int s = (c * NU + v) % kStages;
+      constexpr int kLastRows = (NG & 1) ? kGroupRows : 2 * kGroupRows;
+      const int rows = (v == NU - 1) ? kLastRows : 2 * kGroupRows;   // rows of the unit's tiles
+      // block `warp` of the unit: tile `warp`, [rows][64 B]; rows 64 B apart,
       // so the two rows a quarter-warp reads fall in different bank halves
-      const uint8_t* wb = ring + (size_t)s * kUnitBytes + warp * (kGroupRows * 64);
+      const uint8_t* wb = ring + (size_t)s * kUnitBytes + warp * (rows * 64) + (b & 1) * (kGroupRows * 64);
       const uint4 pa = *reinterpret_cast<const uint4*>(wb + g * 64 + (tig << 4));
       const uint4 pb = *reinterpret_cast<const uint4*>(wb + (g + 8) * 64 + (tig << 4));
       A4[b][0] = pa.x; A4[b][1] = pa.y; A4[b][2] = pa.z; A4[b][3] = pa.w;
@@ -181,20 +173,34 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
     __syncwarp();
     if (lane == 0) {
 #pragma unroll
-      for (int b = 0; b < NG; ++b) mbar_arrive(&wempty[(c * NG + b) % kStages]);
+      for (int v = 0; v < NU; ++v) mbar_arrive(&wempty[(c * NU + v) % kStages]);
     }
     if (!ok) break;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int w = q >> 1, jj = 2 * (q & 1);
+      // codes as the B operand, read per step (they serve every group; held
+      // for the whole chunk they pushed the warp's registers into spilling):
+      // k = 256 * warp + 32 * q + 8 * tig .. + 7 of the chunk -> column tile
+      // 2 * warp + q / 4, 16-byte unit 2 * (q % 4) + tig / 2, half tig % 2
+      uint2 bf[TN];
+#pragma unroll
+      for (int i = 0; i < TN; ++i) {
+        const int m = 8 * i + g;
+        const int unit = (2 * (q & 3) + (tig >> 1)) ^ (m & 7);
+        bf[i] = *reinterpret_cast<const uint2*>(cb + (2 * warp + (q >> 2)) * Lay::kCodeTile + m * 128 + (unit << 4) +
+                                                ((tig & 1) << 3));
+      }
 #pragma unroll
       for (int b = 0; b < NG; ++b) {
         const uint32_t a[4] = {unpack_u8x4(A4[b][w], jj), unpack_u8x4(B4[b][w], jj), unpack_u8x4(A4[b][w], jj + 1),
                                unpack_u8x4(B4[b][w], jj + 1)};
 #pragma unroll
-        for (int i = 0; i < TN; ++i) mma_u8s8_16832(acc[b][SPLIT == 2 ? (q & 1) : i], a, bf[i][q].x, bf[i][q].y);
+        for (int i = 0; i < TN; ++i) mma_u8s8_16832(acc[b][SPLIT == 2 ? (q & 1) : i], a, bf[i].x, bf[i].y);
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&cempty[c & 1]);   // this warp no longer reads the chunk's codes
   }
   if constexpr (SPLIT == 2) {
 #pragma unroll
@@ -225,12 +231,14 @@ HBL_DEVINL bool consume(int nchunks, uint8_t* ring, const uint8_t* cbuf, uint64_
 
 template <int TN, bool OUT_BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __restrict__ codes,
+gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w2, const __grid_constant__ CUtensorMap map_w1,
+                   const __grid_constant__ CUtensorMap map_codes,
                    const int32_t* __restrict__ csum, const float* __restrict__ scales,
                    const float* __restrict__ alpha, int M, int K, int N, uint16_t* __restrict__ Y,
                    int32_t* __restrict__ acc_out) {
   constexpr int MT = 8 * TN;
   using Lay = Layout<MT>;
+  constexpr int kStages = Lay::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = base;
@@ -245,9 +253,11 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __re
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int groups = N / kGroupRows;
   const int G = gridDim.x;
-  const int ng = (groups - (int)blockIdx.x + G - 1) / G;    // groups owned by this CTA
+  const int gbeg = (int)((long long)groups * blockIdx.x / G);          // this CTA's groups: [gbeg, gend)
+  const int ng = (int)((long long)groups * (blockIdx.x + 1) / G) - gbeg;
+  const int nu = (ng + 1) / 2;                                         // weight units per chunk
   const int nchunks = K / kChunk;
-  const int units = nchunks * ng;
+  const int units = nchunks * nu;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -268,17 +278,18 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __re
     if (lane == 0) {
       auto issue_w = [&](int u) {
         const int s = u % kStages;
-        const int c = u / ng, gl = u % ng;
-        const int row0 = ((int)blockIdx.x + gl * G) * kGroupRows;
-        mbar_expect_tx(&wfull[s], kUnitBytes);
-        // 8 blocks x 16 rows x 64 B: eight [16][64 B] tiles in one copy
-        tma_load_3d(ring + (size_t)s * kUnitBytes, &map_w, &wfull[s], 0, row0, c * (kChunk / kKBlock));
+        const int c = u / nu, v = u % nu;
+        const int row0 = (gbeg + 2 * v) * kGroupRows;
+        // 8 blocks x 32 (or 16) rows x 64 B: eight [rows][64 B] tiles in one copy
+        const bool pair = 2 * v + 1 < ng;
+        mbar_expect_tx(&wfull[s], pair ? kUnitBytes : kGroupBytes);
+        tma_load_3d(ring + (size_t)s * kUnitBytes, pair ? &map_w2 : &map_w1, &wfull[s], 0, row0,
+                    c * (kChunk / kKBlock));
       };
       auto issue_c = [&](int c) {
-        uint8_t* dst = cbuf + (size_t)(c & 1) * Lay::kCodeBuf;
-        mbar_expect_tx(&cfull[c & 1], (uint32_t)(M * kChunk));
-        for (int m = 0; m < M; ++m)
-          bulk_load(dst + m * Lay::kCodeRow, codes + (size_t)m * K + (size_t)c * kChunk, kChunk, &cfull[c & 1]);
+        // the whole box counts, zero-filled token rows included
+        mbar_expect_tx(&cfull[c & 1], (uint32_t)Lay::kCodeBuf);
+        tma_load_3d(cbuf + (size_t)(c & 1) * Lay::kCodeBuf, &map_codes, &cfull[c & 1], 0, 0, c * (kChunk / 128));
       };
       int u = 0;
       for (; u < units && u < kStages; ++u) issue_w(u);             // weights do not depend on the previous grid
@@ -286,22 +297,26 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __re
       int issued_c = 0;
       if (nchunks > 0) { issue_c(0); issued_c = 1; }
       bool ok = true;
-      // Codes run one chunk ahead of the weight units: chunk c+1's codes are
-      // requested as soon as the consumers have started chunk c-1 (its buffer
-      // is then free), before chunk c's remaining weight units.
+      // The consumers free chunk c-1's weight slots when they start it (the
+      // fragments are then in registers) and its code buffer when they finish
+      // it. Iteration c therefore first refills weight slots up to chunk c+1
+      // (free since the start of chunk c-1), then chunk c+1's codes (free at
+      // the end of chunk c-1): neither waits behind the other. Blocking waits
+      // (try_wait suspends the thread), so the producer takes no issue slots
+      // from the consumer warps beside it.
       for (int c = 0; c < nchunks && ok; ++c) {
-        if (c + 1 < nchunks) {
+        for (; u < units && u < (c + 2) * nu; ++u) {
+          const int s = u % kStages;
+          if (!mbar_wait(&wempty[s], (uint32_t)((u / kStages) - 1) & 1u, abort)) { ok = false; break; }
+          issue_w(u);
+        }
+        if (ok && c + 1 < nchunks) {
           if (c + 1 >= 2 && !mbar_wait(&cempty[(c + 1) & 1], (uint32_t)(((c + 1) >> 1) - 1) & 1u, abort)) {
             ok = false;
             break;
           }
           issue_c(c + 1);
           issued_c = c + 2;
-        }
-        for (; u < units && u < (c + 1) * ng; ++u) {
-          const int s = u % kStages;
-          if (!mbar_wait(&wempty[s], (uint32_t)((u / kStages) - 1) & 1u, abort)) { ok = false; break; }
-          issue_w(u);
         }
       }
       // bounded drain of the copies issued last
@@ -343,7 +358,7 @@ gemm_stream_kernel(const __grid_constant__ CUtensorMap map_w, const int8_t* __re
     for (int e = threadIdx.x; e < ng * per_group; e += kConsumers * 32) {
       const int gl = e / per_group, rem = e % per_group;
       const int tok = rem / kGroupRows, row = rem % kGroupRows;
-      const int n = ((int)blockIdx.x + gl * G) * kGroupRows + row;
+      const int n = (gbeg + gl) * kGroupRows + row;
       if (tok < M) {
         int s = 0;
 #pragma unroll

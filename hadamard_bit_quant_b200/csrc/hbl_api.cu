@@ -374,15 +374,15 @@ EncodeTiledFn encode_fn() {
 }
 
 // Packed weights viewed as [K/256 blocks][N rows][64 B] (block stride 64 B, row
-// stride K/4 B): one box of [8 blocks][16 rows][64 B] lands as eight
-// consecutive [16][64 B] tiles, the fused decode kernel's unit layout, in one
+// stride K/4 B): one box of [8 blocks][box_rows rows][64 B] lands as eight
+// consecutive [box_rows][64 B] tiles (the decode kernels' unit layout) in one
 // TMA copy.
-bool make_map_w_blocks(CUtensorMap* map, const void* Wpk, int N, int K) {
+bool make_map_w_blocks(CUtensorMap* map, const void* Wpk, int N, int K, int box_rows = 16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)N, (cuuint64_t)K / 256};
   cuuint64_t strides[2] = {(cuuint64_t)K / 4, 64};
-  cuuint32_t box[3] = {64, 16, 8};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 8};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(Wpk), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -470,6 +470,23 @@ int run_gemm_tc(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk, co
                                                                           nullptr, nullptr, acc);
   }
   return launch_status();
+}
+
+// 3-D uint8 tensor map: dims {d0, d1, d2} bytes (d0 contiguous), byte strides {s1, s2}, box {b0, b1, b2}.
+bool make_map_u8_3d(CUtensorMap* map, const void* base, const uint64_t (&dims)[3], const uint64_t (&strides)[2],
+                    const uint32_t (&box)[3], int swizzle_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), d, st, bx, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : (swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE),
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 bool decode_path_fits(int M, int K) {
@@ -589,8 +606,12 @@ int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
                     const float* scales, const float* alpha, uint16_t* Y, int32_t* acc, int sm_count,
                     cudaStream_t s) {
   const int TN = M <= 8 ? 1 : 2;
-  CUtensorMap mw;
-  if (!make_map_w_blocks(&mw, Wpk, N, K)) return -1;
+  CUtensorMap mw2, mw1, mc;
+  if (!make_map_w_blocks(&mw2, Wpk, N, K, 32) || !make_map_w_blocks(&mw1, Wpk, N, K, 16)) return -1;
+  // codes as [K/128 column tiles][M rows][128 B]; one box = one chunk of 2048 k
+  if (!make_map_u8_3d(&mc, codes, {128, (uint64_t)M, (uint64_t)K / 128}, {(uint64_t)K, 128},
+                      {128, (uint32_t)(8 * TN), (uint32_t)(strm::kChunk / 128)}, 128))
+    return -1;
   const int groups = N / strm::kGroupRows;
   const dim3 grid(groups < sm_count ? groups : sm_count);
   ProfScope ps("gemm_decode", s);
@@ -600,12 +621,12 @@ int run_gemm_stream(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
     const size_t sm = strm::Layout<8 * TN_>::kBytes;                                                           \
     if (Y) {                                                                                                   \
       ensure_smem_attr(strm::gemm_stream_kernel<TN_, true>, sm);                                               \
-      e = launch_pdl(strm::gemm_stream_kernel<TN_, true>, grid, dim3(strm::kThreads), sm, s, mw, codes, csum,   \
-                     scales, alpha, M, K, N, Y, (int32_t*)nullptr);                                            \
+      e = launch_pdl(strm::gemm_stream_kernel<TN_, true>, grid, dim3(strm::kThreads), sm, s, mw2, mw1, mc,     \
+                     csum, scales, alpha, M, K, N, Y, (int32_t*)nullptr);                                            \
     } else {                                                                                                   \
       ensure_smem_attr(strm::gemm_stream_kernel<TN_, false>, sm);                                              \
-      e = launch_pdl(strm::gemm_stream_kernel<TN_, false>, grid, dim3(strm::kThreads), sm, s, mw, codes, csum,  \
-                     (const float*)nullptr, (const float*)nullptr, M, K, N, (uint16_t*)nullptr, acc);          \
+      e = launch_pdl(strm::gemm_stream_kernel<TN_, false>, grid, dim3(strm::kThreads), sm, s, mw2, mw1, mc,    \
+                     csum, (const float*)nullptr, (const float*)nullptr, M, K, N, (uint16_t*)nullptr, acc);          \
     }                                                                                                          \
   }
   if (TN == 1) HBL_STRM(1) else HBL_STRM(2)
