@@ -545,6 +545,8 @@ def decode_roofline(torch, hbl, layer, inputs, peaks, peak_kind, steps=20):
     ach = b / t / 1e9
     wbytes = c["N"] * c["K"] / 4
     del g, Wpks
+    floor = launch_floors(torch, int(b), LAYERS)
+    floor["forward_over_read_floor"] = us / floor["read_us"]
     return {"workload": f"decode_oproj M={c['M']} K={c['K']} N={c['N']} W1.58A4 Hon, {LAYERS} weight sets per graph",
             "us_per_forward": us, "tokens_per_s": c["M"] / (us * 1e-6),
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -553,8 +555,49 @@ def decode_roofline(torch, hbl, layer, inputs, peaks, peak_kind, steps=20):
                          "duration_source": ("timed region / launches (CUDA events on the launching stream)"
                                              if single else "CUDA events around each launch, L2 flushed"),
                          "peak_source": f"{peak_kind} hbm_gbs",
-                         "weights_frac": wbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
+                         "weights_frac": wbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                         "single_launch_floor": floor},
             "kernels_cold": prof}
+
+
+def launch_floors(torch, nbytes, sets, reps=20):
+    """What one launch that moves `nbytes` costs on this GPU, measured like the decode forwards
+    (a graph of `sets` launches over `sets` distinct buffers, larger than L2 together, replayed):
+    a reduction that reads the bytes once (torch.sum), and a device-to-device copy of half of them
+    (the same bytes in total, half read and half written). Library kernels, timed only as a floor
+    for the decode rooflines; neither is on the product path."""
+    n32 = nbytes // 4
+    srcs = [torch.randint(-1000, 1000, (n32,), dtype=torch.int32, device="cuda") for _ in range(sets)]
+    dsts = [torch.empty(n32 // 2, dtype=torch.int32, device="cuda") for _ in range(sets)]
+    outs = torch.empty(sets, dtype=torch.int64, device="cuda")
+
+    def graph_us(fn):
+        fn(0)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream()
+        with torch.cuda.graph(g, stream=st):
+            for i in range(sets):
+                fn(i)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / (reps * sets)
+
+    read_us = graph_us(lambda i: torch.sum(srcs[i], dtype=torch.int64, out=outs[i]))
+    copy_us = graph_us(lambda i: dsts[i].copy_(srcs[i][: n32 // 2]))
+    del srcs, dsts
+    torch.cuda.empty_cache()
+    return {"bytes": nbytes, "read_us": read_us, "copy_us": copy_us,
+            "kind": f"graph of {sets} launches over distinct buffers: torch.sum reading the bytes once; "
+                    "device copy of half the bytes (read + written = the bytes)"}
 
 
 def secondary(torch, hbl, layer, inputs):
@@ -588,10 +631,13 @@ def secondary(torch, hbl, layer, inputs):
     g = capture_step(torch, hbl, X, Wpks, wsc, Y, ws, c)
     ms = timed_replays(torch, None, g, 3, 10, 1) / (10 * len(Wpks))
     prof = profile_kernels(torch, hbl, X, Wpks, wsc, Y, ws, c, 16)
+    del g, Wpks
+    floor = launch_floors(torch, big.N * big.K // 4, 16, reps=10)
+    floor["forward_over_read_floor"] = ms * 1e3 / floor["read_us"]
     out["decode M=16 K=16384 N=16384 a4"] = {
         "us_per_forward": ms * 1e3, "tokens_per_s": big.M / (ms * 1e-3),
-        "weight_GBps": big.N * big.K / 4 / (ms * 1e-3) / 1e9, "kernels_cold": prof}
-    del g, Wpks
+        "weight_GBps": big.N * big.K / 4 / (ms * 1e-3) / 1e9, "kernels_cold": prof,
+        "single_launch_floor": floor}
     torch.cuda.empty_cache()
     return out
 
