@@ -20,22 +20,31 @@
 //     rows r*R .. r*R + R - 1, R = ceil(M / CS) <= 2 (256 threads per row,
 //     E = K/256 values per thread, butterflies in registers, passes exchanged
 //     through padded shared memory) into this CTA's shared memory: codes
-//     row-contiguous, scale and per-warp code sums beside them. Lane 0 of
-//     warp q then sends the rows to cluster ranks q and q + 8 (every rank but
-//     this one) with bulk copies (shared memory to distributed shared memory,
-//     completing as transaction bytes on the peer's mbarrier). Each CTA waits
-//     on its own barrier for the M - R rows it receives, so it holds all
-//     M x K codes;
+//     row-contiguous, scale and per-warp code sums beside them. The rows are
+//     then exchanged in one of two ways (flag 16):
+//       - pushed: lane 0 of warp q sends the rows to cluster ranks q and
+//         q + 8 (every rank but this one) with bulk copies (shared memory to
+//         distributed shared memory, completing as transaction bytes on the
+//         peer's mbarrier); each CTA waits on its own barrier for the M - R
+//         rows it receives. Bound by the cluster's copy bandwidth (~30 B/cycle
+//         into each CTA), so it pays at few tokens only;
+//       - through L2: one bulk copy stores this CTA's rows into a global
+//         scratch (the forward's workspace), a cluster barrier orders the
+//         stores before the loads, and one bulk copy brings all M rows back
+//         (every cluster computes the same rows, bit for bit, so clusters that
+//         store to the same scratch store the same bytes).
+//     Either way each CTA then holds all M x K codes;
 //   * the consumers then run the m16n8k32 MMAs of their groups (weights as A,
 //     u = t + 1 unpacked in registers; codes as B), batches of groups
 //     interleaved for independent accumulator chains, add the 8 warps' partial
 //     sums in shared memory, subtract the code sums and store bf16.
-// Two cluster barriers: #1 (arrive at start, wait before the first copy) makes
-// sure every peer runs and has armed its barrier; #2 (arrive once this CTA's
-// rows have all landed, wait at exit) keeps every CTA's shared memory alive
-// until the copies out of it have completed. Every mbarrier wait is bounded;
-// a CTA that gives up sets the device error word, still takes part in both
-// cluster barriers, and writes no output.
+// Two cluster barriers. #1 (arrive at start, wait while X loads) makes sure
+// every peer runs and has armed its barrier. #2: pushed, arrive once this
+// CTA's rows have all landed and wait at exit, which keeps every CTA's shared
+// memory alive until the copies out of it have completed; through L2, arrive
+// once this CTA's rows are in the scratch and wait before loading the others'.
+// Every mbarrier wait is bounded; a CTA that gives up sets the device error
+// word, still takes part in both cluster barriers, and writes no output.
 #pragma once
 #include <cuda.h>
 #include "hbl_common.cuh"
@@ -139,6 +148,25 @@ HBL_DEVINL void bulk_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint
                : "memory");
 }
 HBL_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+// Shared -> global bulk copy of `bytes` (16-byte aligned, multiple of 16),
+// waited for in full (the bytes are written) before the call returns.
+HBL_DEVINL void bulk_store_wait(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(su32(src)), "r"(bytes)
+               : "memory");
+}
+HBL_DEVINL void bulk_commit_wait_all() {
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
+// Global -> shared bulk copy completing as transaction bytes on a local mbarrier.
+HBL_DEVINL void bulk_load_local(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   su32(dst)),
+               "l"(src), "r"(bytes), "r"(su32(bar))
+               : "memory");
+}
+HBL_DEVINL void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;\n" ::: "memory"); }
+
 HBL_DEVINL void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory"); }
 HBL_DEVINL void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory"); }
 HBL_DEVINL void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory"); }
@@ -480,7 +508,7 @@ template <int LOG_K, int TN>
 __global__ void __launch_bounds__(kThreads, 1)
 fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* __restrict__ X, int M, int N,
                     const float* __restrict__ gain, const float* __restrict__ alpha, int flags,
-                    uint16_t* __restrict__ Y) {
+                    uint16_t* __restrict__ Y, uint8_t* __restrict__ xcodes, uint8_t* __restrict__ xmeta) {
   constexpr int MT = 8 * TN;
   using Lay = Layout<LOG_K, MT>;
   constexpr int nchunks = Lay::K / kChunk;
@@ -503,6 +531,7 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
   const int ng = (groups - (int)blockIdx.x + Gd - 1) / Gd;
   const int units = nchunks * ng;
   const bool w3d = (flags & 8) != 0;
+  const bool l2x = (flags & 16) != 0;   // rows exchanged through L2 (else pushed to the peers)
   // token rows [m0, m0 + nr) are transformed and quantised by this CTA:
   // ceil(M / cluster size) rows each (at most kRowBatch, checked at launch)
   const int rpc = (M + (int)csize - 1) / (int)csize;
@@ -515,8 +544,9 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
       mbar_init(&wempty[s], kConsumers);
     }
     mbar_init(codes_full, 1);
-    // every other row arrives from a peer: codes (K bytes) + scale and code sums
-    if (csize > 1) mbar_expect_tx(codes_full, (uint32_t)((M - nr) * (Lay::K + kMetaBytes)));
+    // codes (K bytes) + scale and code sums of every row this CTA receives:
+    // from the peers, the other M - nr rows; from the scratch, all M
+    if (csize > 1) mbar_expect_tx(codes_full, (uint32_t)((l2x ? M : M - nr) * (Lay::K + kMetaBytes)));
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -547,7 +577,7 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
     __syncwarp();
     if (csize > 1) {
       cluster_wait();             // #1
-      cluster_arrive_relaxed();   // #2: the producer receives no rows
+      cluster_arrive_relaxed();   // #2: the producer sends and stores no rows
     }
     if (lane == 0) {
       bool ok = true;
@@ -579,7 +609,7 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
     fence_proxy_async_smem();   // the rows written here are read next by the bulk-copy engine
     consumers_sync();           // ... and by every consumer warp
     bool ok = true;
-    if (csize > 1) {
+    if (csize > 1 && !l2x) {
       // lane 0 of warp w sends to peers w, w + 8 (all peers but this CTA)
       if (lane == 0 && nr > 0) {
         for (uint32_t q = (uint32_t)warp; q < csize; q += kConsumers) {
@@ -594,6 +624,26 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
       // the peers' rows
       ok = __all_sync(0xffffffffu, mbar_wait(codes_full, 0u, abort)) != 0;
       cluster_arrive_relaxed();   // #2: every row this CTA receives has landed
+    } else if (csize > 1) {
+      // this CTA's rows -> the scratch, written in full before barrier #2
+      if (warp == 0 && lane == 0 && nr > 0) {
+        const uint32_t cb_off = (uint32_t)m0 * Lay::K, mt_off = (uint32_t)m0 * kMetaBytes;
+        bulk_store_wait(xcodes + cb_off, cbuf + cb_off, (uint32_t)nr * Lay::K);
+        bulk_store_wait(xmeta + mt_off, reinterpret_cast<uint8_t*>(meta) + mt_off, (uint32_t)nr * kMetaBytes);
+        bulk_commit_wait_all();
+        fence_proxy_async_global();
+      }
+      __syncwarp();
+      cluster_arrive_release();   // #2: this CTA's rows are in the scratch
+      cluster_wait();
+      // every row of the cluster is in the scratch: load all M of them (this
+      // CTA's own rows come back unchanged)
+      if (warp == 0 && lane == 0) {
+        fence_proxy_async_global();
+        bulk_load_local(cbuf, xcodes, (uint32_t)M * Lay::K, codes_full);
+        bulk_load_local(meta, xmeta, (uint32_t)M * kMetaBytes, codes_full);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(codes_full, 0u, abort)) != 0;
     }
 
     // ----- consumers, phase 2: MMAs over the weight ring -----
@@ -630,9 +680,9 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap map_w, const uint16_t* _
         }
       }
     }
-    // #2: every copy into every CTA of the cluster has landed, so the rows this
-    // CTA sent have been read and its shared memory may be released
-    if (csize > 1) cluster_wait();
+    // pushed: #2, every copy into every CTA of the cluster has landed, so the
+    // rows this CTA sent have been read and its shared memory may be released
+    if (csize > 1 && !l2x) cluster_wait();
   }
 }
 

@@ -671,6 +671,10 @@ int run_gemm_decode(const int8_t* codes, int M, int K, int N, const uint8_t* Wpk
 // Fused single-kernel decode forward (1..16 tokens, K in {2048, 4096, 8192}).
 // ---------------------------------------------------------------------------
 constexpr int kFusedNotApplicable = -1;
+#ifndef HBL_FUSED_L2_CLUSTER
+#define HBL_FUSED_L2_CLUSTER 16
+#endif
+constexpr int kFusedL2Cluster = HBL_FUSED_L2_CLUSTER;   // smallest cluster exchanging rows through L2
 
 // Preferred cluster size of the fused decode kernel: one token row per CTA,
 // i.e. M rounded up to a power of two (16-CTA clusters are non-portable and
@@ -687,7 +691,7 @@ int fused_cluster_size(int M) {
 
 template <int LOG_K, int TN>
 int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const float* gain, const float* alpha,
-                 int flags, uint16_t* Y, int sm_count, cudaStream_t s) {
+                 int flags, uint16_t* Y, uint8_t* xcodes, uint8_t* xmeta, int sm_count, cudaStream_t s) {
   auto* kern = fdec::fused_decode_kernel<LOG_K, TN>;
   const size_t smem = fdec::Layout<LOG_K, 8 * TN>::kBytes;
   ensure_smem_attr(kern, smem);
@@ -736,8 +740,12 @@ int launch_fused(const CUtensorMap& mw, const uint16_t* X, int M, int N, const f
   }
   attr[0].val.clusterDim.x = (unsigned)CS;
   cfg.gridDim = dim3((unsigned)grid);
+  // rows exchanged through L2 in 16-CTA clusters (measured on B200, M=16:
+  // 8.7 -> 7.1 us), pushed through distributed shared memory in smaller ones
+  // (M=4: 5.0 us pushed, 5.4 us through L2)
+  if (CS >= kFusedL2Cluster) flags |= 16;
   ProfScope ps("fused_decode", s);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, X, M, N, gain, alpha, flags, Y);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mw, X, M, N, gain, alpha, flags, Y, xcodes, xmeta);
   return e == cudaSuccess ? launch_status() : HBL_ERR_CUDA;
 }
 
@@ -748,8 +756,11 @@ bool fused_fits(int M, int K, int N) {
   return (long long)MT * K <= 65536;
 }
 
+// xcodes (M x K bytes) and xmeta (M x 48 bytes), 16-byte aligned: the global
+// scratch through which the CTAs of a cluster exchange their token rows.
 int run_fused_decode(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, const float* wscale, int act_bits,
-                     int use_hadamard, bool ln, const float* gain, uint16_t* Y, int sm_count, cudaStream_t s) {
+                     int use_hadamard, bool ln, const float* gain, uint16_t* Y, uint8_t* xcodes, uint8_t* xmeta,
+                     int sm_count, cudaStream_t s) {
   // [16 rows][64 B] tiles, unswizzled (the fused kernel's conflict-free fragment
   // reads): one 3-D copy per 8 KB unit where the driver accepts the blocked
   // view, else eight 2-D copies
@@ -762,11 +773,11 @@ int run_fused_decode(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk,
   }
   const bool tn1 = M <= 8;
   switch (K) {
-    case 2048: return tn1 ? launch_fused<11, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
-                          : launch_fused<11, 2>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s);
-    case 4096: return tn1 ? launch_fused<12, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
-                          : launch_fused<12, 2>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s);
-    case 8192: return tn1 ? launch_fused<13, 1>(mw, X, M, N, gain, wscale, flags, Y, sm_count, s)
+    case 2048: return tn1 ? launch_fused<11, 1>(mw, X, M, N, gain, wscale, flags, Y, xcodes, xmeta, sm_count, s)
+                          : launch_fused<11, 2>(mw, X, M, N, gain, wscale, flags, Y, xcodes, xmeta, sm_count, s);
+    case 4096: return tn1 ? launch_fused<12, 1>(mw, X, M, N, gain, wscale, flags, Y, xcodes, xmeta, sm_count, s)
+                          : launch_fused<12, 2>(mw, X, M, N, gain, wscale, flags, Y, xcodes, xmeta, sm_count, s);
+    case 8192: return tn1 ? launch_fused<13, 1>(mw, X, M, N, gain, wscale, flags, Y, xcodes, xmeta, sm_count, s)
                           : kFusedNotApplicable;
     default: return kFusedNotApplicable;
   }
@@ -784,7 +795,11 @@ int forward_impl(const uint16_t* X, int M, int K, int N, const uint8_t* Wpk, con
   int32_t* D = reinterpret_cast<int32_t*>(base + L.dacc);
   const int path = g_gemm_path.load(std::memory_order_relaxed);
   if ((path == 0 || path == 6) && fused_fits(M, K, N)) {
-    const int fs = run_fused_decode(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, ln, gain, Y, d->sm_count, s);
+    // the exchange scratch: the codes region (M x K) and the accumulator
+    // region (M x N x 4 >= M x 48 bytes), neither used by the fused path otherwise
+    static_assert(fdec::kMetaBytes <= 4 * fdec::kGroupRows, "row metadata fits the accumulator region");
+    const int fs = run_fused_decode(X, M, K, N, Wpk, wscale, act_bits, use_hadamard, ln, gain, Y,
+                                    reinterpret_cast<uint8_t*>(codes), reinterpret_cast<uint8_t*>(D), d->sm_count, s);
     if (fs != kFusedNotApplicable) return fs;
   }
   int st = run_quantize(X, M, K, act_bits, use_hadamard, codes, scales, csum, s, ln, gain);
