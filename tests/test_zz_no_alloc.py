@@ -29,7 +29,7 @@ def H():
 
 CASES = [
     # M, K, N, act_bits, use_hadamard, GEMM path (0 = by size, 1 = warp-level split-K)
-    (16, 4096, 4096, 4, 1, 0),     # decode-shaped o_proj, W1.58A4 (fused kernel: no workspace use)
+    (16, 4096, 4096, 4, 1, 0),     # decode-shaped o_proj, W1.58A4 (fused kernel: token rows exchanged through the workspace)
     (3, 1024, 256, 8, 0, 0),       # plain BitLinear, INT8
     (100, 4096, 512, 4, 1, 1),     # split-K: codes, scales and int32 partials all live in the workspace
     (200, 2048, 1024, 8, 1, 2),    # persistent tcgen05 GEMM reading codes from the workspace
